@@ -1,0 +1,162 @@
+/*
+ * lite_attn.h -- C ABI of the B200 (sm_100a) LiteAttention forward pass.
+ *
+ * LiteAttention ("LiteAttention: A Temporal Sparse Attention for Diffusion Transformers",
+ * arXiv 2511.11062; README of moonmath-ai/LiteAttention) is FlashAttention-style softmax
+ * self-attention that reads a persistent per-(batch, head, query tile, key tile) Skip-Mask,
+ * bypasses every marked tile completely (no QK^T, no softmax, no PV, no K/V load: README,
+ * "Full-Stage Elimination"), and on every tile it does compute evaluates the QK-Skip test inside
+ * the online softmax (README, "QK-Skip Algorithm"; skill page "Lite Attention Temporal Sparse",
+ * Core Concept). Tiles that pass the test are OR-ed into the mask for the next denoising step,
+ * so the mask only grows.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All functions are extern "C", return an int status (LITE_OK = 0, negative = error) and never
+ *    throw. Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream) and the
+ *    call returns after enqueueing; nothing synchronises except lite_get_device_status().
+ *  - Every buffer is owned by the caller, who allocates and frees it; the library keeps no state
+ *    between calls (one mask pair per attention layer, README: separate instances per layer).
+ *    Device pointers must be device-accessible memory of the current device.
+ *  - Layouts:
+ *      q, k, v, o : bf16 [B, N, H, d], contiguous, 16-byte aligned. The output o viewed as
+ *                   [B, N, H*d] is the README's (batch, seq_len, heads*head_dim) return layout.
+ *      lse        : fp32 [B, H, N], natural log of the softmax normaliser of each query row.
+ *      masks      : uint32 [B, H, T, W]. Bit (j & 31) of word (j >> 5) set = skip key tile j for
+ *                   that (b, h, query tile). T = ceil(N / tile), W = ceil(T / 32). Bits at or
+ *                   above T in the last word are ignored and written as 0.
+ *      tile       : 64 for d = 64, 128 for d = 128 (lite_mask_geometry reports it).
+ *  - Argument errors are reported before any CUDA call is made.
+ */
+#ifndef LITE_ATTN_H
+#define LITE_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without pulling in the CUDA headers. */
+typedef struct CUstream_st* lite_stream_t;
+
+enum {
+  LITE_OK = 0,
+  LITE_ERR_INVALID_ARG = -1, /* NULL required pointer, B/H/N <= 0, NaN tau, tau > 0 outside debug */
+  LITE_ERR_UNSUPPORTED = -2, /* d not in {64, 128}, misaligned pointer, T or sizes beyond limits  */
+  LITE_ERR_CUDA = -3,        /* a CUDA launch, allocation or query failed                          */
+  LITE_ERR_TIMEOUT = -4,     /* device status: a kernel wait exceeded its time limit and gave up   */
+  LITE_ERR_CHECK = -5        /* device status: an in-kernel consistency check failed               */
+};
+
+/*
+ * lite_attn_fwd -- one LiteAttention forward for one layer at one denoising step.
+ *
+ * Computes, for every (b, h) and query row n, o = softmax(scale * q k^T) v over the key tiles that
+ * mask_in leaves live (README, "Full-Stage Elimination"), and lse = log-sum-exp of those scores
+ * (README: LSE is returned for combining partial attentions). While doing so it runs the QK-Skip
+ * test on every computed tile: the key tiles of a query tile are visited from the highest index
+ * down (README, must_do_list: "we iterate in reverse order inside of the kernel"); with m_r the
+ * running row maximum of scale*QK^T over the tiles visited before tile j and loc_r the row maximum
+ * inside tile j, tile j is flagged when loc_r - m_r < tau for every valid row r of the query tile.
+ * mask_out = mask_in | flags (README, "QK-Skip Algorithm": the number of skipped tiles only grows).
+ *
+ *  q, k, v    in   device bf16 [B, N, H, d].
+ *  o          out  device bf16 [B, N, H, d].
+ *  lse        out  device fp32 [B, H, N], or NULL to skip writing it.
+ *  mask_in    in   device uint32 [B, H, T, W], or NULL = nothing skipped (fresh state, README
+ *                  reset_skip_state()).
+ *  mask_out   out  device uint32 [B, H, T, W], or NULL = do not record flags. It may equal
+ *                  mask_in (in place); otherwise the library first copies mask_in into it.
+ *  B, H, N, d      batch, heads, tokens, head dim (d in {64, 128}); T = ceil(N/tile) <= 4096.
+ *  scale           softmax scale; <= 0 or NaN selects 1/sqrt(d) (README's Wan2.1 call omits it).
+ *  tau             QK-Skip threshold in natural-log units of scale*QK^T (README: default -10;
+ *                  -6, -3, 0 in its examples). -inf disables flagging. tau > 0 is refused unless
+ *                  the environment variable LITE_ATTN_DEBUG is set to anything but "FALSE"
+ *                  (README: LITE_ATTENTION_DEBUG). NaN is refused.
+ *  stream          CUDA stream for all work.
+ *
+ * A query tile whose live list is empty (only possible with a caller-built mask) yields o = 0 and
+ * lse = -inf for its rows. Scratch memory (per-row live lists and the work order) is taken with
+ * cudaMallocAsync on `stream` and released with cudaFreeAsync on the same stream.
+ * Returns LITE_OK once enqueued; device-side failures are reported by lite_get_device_status().
+ */
+int lite_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const uint32_t* mask_in, uint32_t* mask_out, int B, int H, int N, int d,
+                  float scale, float tau, lite_stream_t stream);
+
+/*
+ * lite_attn_dense -- the no-skip path (README: turning skipping off "falls back to regular FA3").
+ *
+ * Same kernel and layouts as lite_attn_fwd with every tile live and the QK-Skip test off; no mask
+ * is read or written and no scratch memory is allocated. lse may be NULL.
+ */
+int lite_attn_dense(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                    int N, int d, float scale, lite_stream_t stream);
+
+/*
+ * lite_mask_to_list -- Skip-Mask to Skip-List compaction (skill page, Architecture Overview:
+ * "Bitmask (or Skip-List for high sparsity)"; README: key ranges are iterated in reverse order).
+ *
+ *  mask    in   device uint32 [B, H, T, W], or NULL = nothing skipped.
+ *  list    out  device int16 [B, H, T, T]: for each (b, h, query tile) the live key tiles in
+ *               descending order in the first counts[...] entries; later entries are untouched.
+ *  counts  out  device int32 [B, H, T]: number of live key tiles per query tile.
+ *  B, H, N, d   as in lite_attn_fwd (they fix T and W).
+ */
+int lite_mask_to_list(const uint32_t* mask, int16_t* list, int32_t* counts, int B, int H, int N,
+                      int d, lite_stream_t stream);
+
+/*
+ * lite_schedule -- work order for the persistent attention kernel (no counterpart on the pages;
+ * it orders the query tiles that lite_attn_fwd processes).
+ *
+ * Heads (b, h) are ordered by decreasing total live-tile count (ties: lower b*H+h first); inside a
+ * head, query tiles by decreasing live count (ties: lower index first). Writes order[B*H*T] with
+ * entries (b*H + h)*T + i: a longest-first list schedule that keeps one head's query tiles
+ * together so that concurrently running tiles share K/V in L2.
+ *
+ *  counts  in   device int32 [B, H, T] (from lite_mask_to_list), each in [0, T].
+ *  order   out  device int32 [B*H*T].
+ *  B*H <= 8192 and T <= 4096 (LITE_ERR_UNSUPPORTED otherwise).
+ */
+int lite_schedule(const int32_t* counts, int32_t* order, int B, int H, int T, lite_stream_t stream);
+
+/* Host only: tile edge, tiles per side and mask words per row for (N, d). */
+int lite_mask_geometry(int N, int d, int* tile, int* T, int* words);
+
+/*
+ * lite_get_device_status -- synchronises `stream`, then reads and clears the device status word of
+ * the current device. Returns LITE_OK, LITE_ERR_TIMEOUT (a kernel wait gave up after its time
+ * limit; that call's outputs are invalid), LITE_ERR_CHECK, or LITE_ERR_CUDA if the stream itself
+ * reports an error.
+ */
+int lite_get_device_status(lite_stream_t stream);
+
+/* Static description of a status code; never NULL. */
+const char* lite_status_string(int status);
+
+/*
+ * Process-wide options (host state, not thread-safe against concurrent launches):
+ *  LITE_OPT_WAIT_LIMIT_NS  upper bound, in nanoseconds, on any single in-kernel wait before the
+ *                          kernel gives up and reports LITE_ERR_TIMEOUT (default 4e9; >= 1000).
+ *  LITE_OPT_DEBUG_STALL    1 = test hook: the MMA warp of every CTA withholds its first tile, so
+ *                          the waits that depend on it run out their limit (no fault, no hang).
+ *  LITE_OPT_MAX_CTAS       cap on the persistent grid size (0 = one CTA per SM).
+ * Returns LITE_ERR_INVALID_ARG for an unknown option or out-of-range value.
+ */
+enum { LITE_OPT_WAIT_LIMIT_NS = 1, LITE_OPT_DEBUG_STALL = 2, LITE_OPT_MAX_CTAS = 3 };
+int lite_set_option(int option, long long value);
+
+/*
+ * lite_set_kernel_events -- measurement hook. While set, every lite_attn_fwd / lite_attn_dense
+ * call records `before` immediately before and `after` immediately after its attention kernel, on
+ * the call's stream. Both are cudaEvent_t handles owned by the caller; pass NULL, NULL to stop.
+ */
+int lite_set_kernel_events(void* before, void* after);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LITE_ATTN_H */

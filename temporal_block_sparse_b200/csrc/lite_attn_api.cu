@@ -1,0 +1,326 @@
+// lite_attn_api.cu -- host side of the C ABI declared in include/lite_attn.h.
+//
+// Validates arguments (before any CUDA call), builds the TMA tensor maps, takes stream-ordered
+// scratch memory and enqueues: compaction (Skip-Mask -> Skip-List, mask copy) -> schedule (LPT
+// work order) -> persistent attention. Status words, options and per-device caches live here.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "attn_kernel.cuh"
+#include "lite_attn.h"
+#include "mask_kernels.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxT = 4096;
+
+__device__ int g_device_status;  // one per device; set by kernels, read/cleared by the host
+
+struct Options {
+  unsigned long long wait_limit_ns = 4000000000ull;
+  int debug_stall = 0;
+  int max_ctas = 0;
+};
+Options g_opt;
+cudaEvent_t g_ev_before = nullptr;
+cudaEvent_t g_ev_after = nullptr;
+
+struct DeviceCache {
+  bool init = false;
+  int sms = 0;
+  int* status = nullptr;
+  bool smem_set[4] = {false, false, false, false};
+};
+DeviceCache g_dev[kMaxDevices];
+std::mutex g_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+cudaStream_t as_stream(lite_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int device_cache(DeviceCache** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LITE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceCache& c = g_dev[dev];
+  if (!c.init) {
+    if (cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return LITE_ERR_CUDA;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&c.status), g_device_status) != cudaSuccess)
+      return LITE_ERR_CUDA;
+    c.init = true;
+  }
+  if (!g_encode) {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return LITE_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  *out = &c;
+  return LITE_OK;
+}
+
+bool debug_env() {
+  const char* e = std::getenv("LITE_ATTN_DEBUG");
+  return e && std::strcmp(e, "FALSE") != 0;
+}
+
+int tile_for(int d) { return d == 64 ? 64 : (d == 128 ? 128 : 0); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shapes(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0) return LITE_ERR_INVALID_ARG;
+  const int t = tile_for(d);
+  if (!t) return LITE_ERR_UNSUPPORTED;
+  const long long T = (static_cast<long long>(N) + t - 1) / t;
+  if (T > kMaxT) return LITE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * T > (1ll << 30)) return LITE_ERR_UNSUPPORTED;
+  return LITE_OK;
+}
+
+int check_qkvo(const void* q, const void* k, const void* v, const void* o, const float* lse) {
+  if (!q || !k || !v || !o) return LITE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LITE_ERR_UNSUPPORTED;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LITE_ERR_UNSUPPORTED;
+  return LITE_OK;
+}
+
+// [B, N, H, d] bf16 viewed as a 4-D tensor (d, H, N, B); box = 64 elements x 1 head x rows x 1.
+bool make_tmap(CUtensorMap* map, const void* ptr, int B, int N, int H, int d, int rows) {
+  cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(H), cuuint64_t(N), cuuint64_t(B)};
+  cuuint64_t strides[3] = {cuuint64_t(d) * 2, cuuint64_t(H) * d * 2, cuuint64_t(N) * H * d * 2};
+  cuuint32_t box[4] = {64, 1, cuuint32_t(rows), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+float resolve_scale(float scale, int d) {
+  if (!(scale > 0.f) || std::isnan(scale)) return 1.0f / std::sqrt(static_cast<float>(d));
+  return scale;
+}
+
+template <int D, int BN>
+int launch_attention(DeviceCache* dc, int cfg_slot, const void* q, const void* k, const void* v,
+                     lite::AttnParams p, cudaStream_t stream) {
+  using C = lite::AttnCfg<D, BN>;
+  if (!dc->smem_set[cfg_slot]) {
+    if (cudaFuncSetAttribute(lite::lite_attn_kernel<D, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess)
+      return LITE_ERR_CUDA;
+    dc->smem_set[cfg_slot] = true;
+  }
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, p.B, p.N, p.H, D, C::BQ) || !make_tmap(&tk, k, p.B, p.N, p.H, D, BN) ||
+      !make_tmap(&tv, v, p.B, p.N, p.H, D, BN))
+    return LITE_ERR_CUDA;
+  int grid = dc->sms;
+  if (g_opt.max_ctas > 0 && g_opt.max_ctas < grid) grid = g_opt.max_ctas;
+  if (p.n_items < grid) grid = p.n_items;
+  if (grid <= 0) return LITE_OK;
+  if (g_ev_before) cudaEventRecord(g_ev_before, stream);
+  lite::lite_attn_kernel<D, BN><<<grid, 192, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
+  if (g_ev_after) cudaEventRecord(g_ev_after, stream);
+  return LITE_OK;
+}
+
+int run_attention(DeviceCache* dc, int d, const void* q, const void* k, const void* v, const lite::AttnParams& p,
+                  cudaStream_t stream) {
+  if (d == 64) return launch_attention<64, 64>(dc, 0, q, k, v, p, stream);
+  return launch_attention<128, 128>(dc, 1, q, k, v, p, stream);
+}
+
+lite::AttnParams base_params(void* o, float* lse, int B, int H, int N, int d, float scale, DeviceCache* dc) {
+  lite::AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int t = tile_for(d);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.T = (N + t - 1) / t;
+  p.W = (p.T + 31) / 32;
+  p.n_items = B * H * p.T;
+  p.scale_log2 = resolve_scale(scale, d) * 1.4426950408889634f;
+  p.tau_log2 = -INFINITY;
+  p.status = dc->status;
+  p.wait_limit_ns = g_opt.wait_limit_ns;
+  p.debug_stall = g_opt.debug_stall;
+  return p;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+extern "C" {
+
+int lite_mask_geometry(int N, int d, int* tile, int* T, int* words) {
+  if (N <= 0) return LITE_ERR_INVALID_ARG;
+  const int t = tile_for(d);
+  if (!t) return LITE_ERR_UNSUPPORTED;
+  const int TT = (N + t - 1) / t;
+  if (tile) *tile = t;
+  if (T) *T = TT;
+  if (words) *words = (TT + 31) / 32;
+  return LITE_OK;
+}
+
+const char* lite_status_string(int status) {
+  switch (status) {
+    case LITE_OK: return "ok";
+    case LITE_ERR_INVALID_ARG: return "invalid argument";
+    case LITE_ERR_UNSUPPORTED: return "unsupported shape, head dim or alignment";
+    case LITE_ERR_CUDA: return "CUDA launch, allocation or query failed";
+    case LITE_ERR_TIMEOUT: return "a kernel wait exceeded its time limit; outputs of that call are invalid";
+    case LITE_ERR_CHECK: return "an in-kernel consistency check failed";
+    default: return "unknown status";
+  }
+}
+
+int lite_set_option(int option, long long value) {
+  switch (option) {
+    case LITE_OPT_WAIT_LIMIT_NS:
+      if (value < 1000) return LITE_ERR_INVALID_ARG;
+      g_opt.wait_limit_ns = static_cast<unsigned long long>(value);
+      return LITE_OK;
+    case LITE_OPT_DEBUG_STALL:
+      if (value != 0 && value != 1) return LITE_ERR_INVALID_ARG;
+      g_opt.debug_stall = static_cast<int>(value);
+      return LITE_OK;
+    case LITE_OPT_MAX_CTAS:
+      if (value < 0 || value > 1000000) return LITE_ERR_INVALID_ARG;
+      g_opt.max_ctas = static_cast<int>(value);
+      return LITE_OK;
+    default:
+      return LITE_ERR_INVALID_ARG;
+  }
+}
+
+int lite_set_kernel_events(void* before, void* after) {
+  if ((before == nullptr) != (after == nullptr)) return LITE_ERR_INVALID_ARG;
+  g_ev_before = static_cast<cudaEvent_t>(before);
+  g_ev_after = static_cast<cudaEvent_t>(after);
+  return LITE_OK;
+}
+
+int lite_get_device_status(lite_stream_t stream) {
+  DeviceCache* dc = nullptr;
+  if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return LITE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, dc->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return LITE_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(dc->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return LITE_ERR_CUDA;
+  }
+  return v;
+}
+
+int lite_mask_to_list(const uint32_t* mask, int16_t* list, int32_t* counts, int B, int H, int N, int d,
+                      lite_stream_t stream) {
+  if (!list || !counts) return LITE_ERR_INVALID_ARG;
+  int st = check_shapes(B, H, N, d);
+  if (st) return st;
+  DeviceCache* dc = nullptr;
+  if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
+  const int t = tile_for(d), T = (N + t - 1) / t, W = (T + 31) / 32;
+  const int rows = B * H * T;
+  lite::lite_compact_kernel<<<(rows + 7) / 8, 256, 0, as_stream(stream)>>>(mask, nullptr, list, counts, rows, T, W);
+  return cudaGetLastError() == cudaSuccess ? LITE_OK : LITE_ERR_CUDA;
+}
+
+int lite_schedule(const int32_t* counts, int32_t* order, int B, int H, int T, lite_stream_t stream) {
+  if (!counts || !order || B <= 0 || H <= 0 || T <= 0) return LITE_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 8192 || T > kMaxT) return LITE_ERR_UNSUPPORTED;
+  DeviceCache* dc = nullptr;
+  if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
+  const int BH = B * H;
+  const size_t sm = size_t(BH + T) * sizeof(int32_t);
+  lite::lite_schedule_kernel<<<BH, 512, sm, as_stream(stream)>>>(counts, order, BH, T);
+  return cudaGetLastError() == cudaSuccess ? LITE_OK : LITE_ERR_CUDA;
+}
+
+int lite_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const uint32_t* mask_in,
+                  uint32_t* mask_out, int B, int H, int N, int d, float scale, float tau, lite_stream_t stream) {
+  int st = check_qkvo(q, k, v, o, lse);
+  if (st) return st;
+  st = check_shapes(B, H, N, d);
+  if (st) return st;
+  if (std::isnan(tau)) return LITE_ERR_INVALID_ARG;
+  if (tau > 0.f && !debug_env()) return LITE_ERR_INVALID_ARG;
+  if ((mask_in && (reinterpret_cast<uintptr_t>(mask_in) & 3u)) || (mask_out && (reinterpret_cast<uintptr_t>(mask_out) & 3u)))
+    return LITE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > 8192) return LITE_ERR_UNSUPPORTED;
+  DeviceCache* dc = nullptr;
+  if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  lite::AttnParams p = base_params(o, lse, B, H, N, d, scale, dc);
+  const int T = p.T, W = p.W, rows = p.n_items;
+
+  // scratch: live lists, counts, order, work counter
+  const size_t list_b = align256(size_t(rows) * T * sizeof(int16_t));
+  const size_t cnt_b = align256(size_t(rows) * sizeof(int32_t));
+  const size_t ord_b = align256(size_t(rows) * sizeof(int32_t));
+  const size_t total = list_b + 2 * cnt_b + 256;
+  void* ws = nullptr;
+  if (cudaMallocAsync(&ws, total, s) != cudaSuccess) return LITE_ERR_CUDA;
+  char* base = static_cast<char*>(ws);
+  int16_t* list = reinterpret_cast<int16_t*>(base);
+  int32_t* counts = reinterpret_cast<int32_t*>(base + list_b);
+  int32_t* order = reinterpret_cast<int32_t*>(base + list_b + cnt_b);
+  int32_t* counter = reinterpret_cast<int32_t*>(base + list_b + cnt_b + ord_b);
+  (void)ord_b;
+
+  st = LITE_OK;
+  if (cudaMemsetAsync(counter, 0, sizeof(int32_t), s) != cudaSuccess) st = LITE_ERR_CUDA;
+  if (!st) {
+    lite::lite_compact_kernel<<<(rows + 7) / 8, 256, 0, s>>>(mask_in, mask_out, list, counts, rows, T, W);
+    if (cudaGetLastError() != cudaSuccess) st = LITE_ERR_CUDA;
+  }
+  if (!st) {
+    const size_t sm = size_t(B * H + T) * sizeof(int32_t);
+    lite::lite_schedule_kernel<<<B * H, 512, sm, s>>>(counts, order, B * H, T);
+    if (cudaGetLastError() != cudaSuccess) st = LITE_ERR_CUDA;
+  }
+  if (!st) {
+    p.mask_out = mask_out;
+    p.list = list;
+    p.counts = counts;
+    p.order = order;
+    p.work_counter = counter;
+    p.tau_log2 = tau * 1.4426950408889634f;
+    p.skip_test = (mask_out != nullptr && tau > -INFINITY) ? 1 : 0;
+    st = run_attention(dc, d, q, k, v, p, s);
+  }
+  if (cudaFreeAsync(ws, s) != cudaSuccess && !st) st = LITE_ERR_CUDA;
+  return st;
+}
+
+int lite_attn_dense(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                    float scale, lite_stream_t stream) {
+  int st = check_qkvo(q, k, v, o, lse);
+  if (st) return st;
+  st = check_shapes(B, H, N, d);
+  if (st) return st;
+  DeviceCache* dc = nullptr;
+  if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
+  lite::AttnParams p = base_params(o, lse, B, H, N, d, scale, dc);
+  // every tile live, identity order, static striding over items (uniform cost): no scratch
+  return run_attention(dc, d, q, k, v, p, as_stream(stream));
+}
+
+}  // extern "C"

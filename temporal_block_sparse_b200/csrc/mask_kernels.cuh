@@ -1,0 +1,79 @@
+// mask_kernels.cuh -- Skip-Mask bookkeeping on the device.
+//
+//  * lite_compact_kernel: Skip-Mask -> Skip-List. One warp per (b, h, query tile). The mask row is
+//    read one 32-bit word at a time from the top word down; lane l owns key tile 32*w + 31 - l, so a
+//    ballot plus a prefix popcount gives every live tile its slot in descending order (the README's
+//    reverse iteration order). The same pass copies the row into mask_out (with bits >= T cleared),
+//    which is where the attention kernel later ORs new flags.
+//  * lite_schedule_kernel: one CTA per head. Ranks the head among all heads by total live work,
+//    then places each of its query tiles by (live count desc, index asc) with an O(T^2) rank count
+//    in shared memory -- deterministic, no atomics on the output.
+#pragma once
+
+#include <stdint.h>
+
+namespace lite {
+
+// mask_in may alias mask_out (in-place update): each warp reads a word before it writes it back.
+__global__ void __launch_bounds__(256) lite_compact_kernel(const uint32_t* mask_in,
+                                                          uint32_t* mask_out, int16_t* __restrict__ list,
+                                                          int32_t* __restrict__ counts, int rows, int T,
+                                                          int W) {
+  const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp_global >= rows) return;
+  const size_t row = size_t(warp_global);
+  const uint32_t tail_mask = (T & 31) ? ((1u << (T & 31)) - 1u) : 0xffffffffu;
+  int count = 0;
+  for (int w = W - 1; w >= 0; --w) {
+    uint32_t word = mask_in ? mask_in[row * W + w] : 0u;
+    if (w == W - 1) word &= tail_mask;  // bits >= T carry no tile
+    if (mask_out && lane == 0) mask_out[row * W + w] = word;
+    const int j = w * 32 + 31 - lane;
+    const bool live = (j < T) && !((word >> (31 - lane)) & 1u);
+    const uint32_t bal = __ballot_sync(0xffffffffu, live);
+    if (live && list) list[row * T + count + __popc(bal & ((1u << lane) - 1u))] = int16_t(j);
+    count += __popc(bal);
+  }
+  if (lane == 0) counts[row] = count;
+}
+
+// smem: totals[BH] ints, then counts of this head [T] ints
+__global__ void __launch_bounds__(512) lite_schedule_kernel(const int32_t* __restrict__ counts,
+                                                           int32_t* __restrict__ order, int BH, int T) {
+  extern __shared__ int32_t sh[];
+  int32_t* totals = sh;
+  int32_t* mine = sh + BH;
+  const int g = blockIdx.x;
+  for (int x = threadIdx.x; x < BH; x += blockDim.x) totals[x] = 0;
+  __syncthreads();
+  // per-head totals (every CTA computes all of them; B*H*T ints, served from L2)
+  for (int x = threadIdx.x; x < BH * T; x += blockDim.x) {
+    const int v = __ldg(counts + x);
+    if (v) atomicAdd(&totals[x / T], v);
+  }
+  for (int x = threadIdx.x; x < T; x += blockDim.x) mine[x] = __ldg(counts + size_t(g) * T + x);
+  __syncthreads();
+  // rank of this head: heads with more work, or equal work and a lower index, go first
+  const int my_total = totals[g];
+  __shared__ int rank_acc;
+  if (threadIdx.x == 0) rank_acc = 0;
+  __syncthreads();
+  int before = 0;
+  for (int x = threadIdx.x; x < BH; x += blockDim.x)
+    before += (totals[x] > my_total) || (totals[x] == my_total && x < g);
+  atomicAdd(&rank_acc, before);
+  __syncthreads();
+  const size_t base = size_t(rank_acc) * T;
+  for (int i = threadIdx.x; i < T; i += blockDim.x) {
+    const int c = mine[i];
+    int pos = 0;
+    for (int x = 0; x < T; ++x) {
+      const int cx = mine[x];
+      pos += (cx > c) || (cx == c && x < i);
+    }
+    order[base + pos] = g * T + i;
+  }
+}
+
+}  // namespace lite

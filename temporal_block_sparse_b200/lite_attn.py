@@ -1,0 +1,186 @@
+"""Python binding of the LiteAttention C ABI (include/lite_attn.h).
+
+Argument marshalling only: every step of the forward pass runs in the CUDA library
+`liblite_attn.so` built next to this file. There is no fallback -- if the library is missing or
+cannot be loaded, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblite_attn.so")
+
+LITE_OK = 0
+LITE_ERR_INVALID_ARG = -1
+LITE_ERR_UNSUPPORTED = -2
+LITE_ERR_CUDA = -3
+LITE_ERR_TIMEOUT = -4
+LITE_ERR_CHECK = -5
+
+LITE_OPT_WAIT_LIMIT_NS = 1
+LITE_OPT_DEBUG_STALL = 2
+LITE_OPT_MAX_CTAS = 3
+
+# every exported symbol and its (argtypes, restype)
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+SIGNATURES = {
+    "lite_attn_fwd": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _F, _P], _I),
+    "lite_attn_dense": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P], _I),
+    "lite_mask_to_list": ([_P, _P, _P, _I, _I, _I, _I, _P], _I),
+    "lite_schedule": ([_P, _P, _I, _I, _I, _P], _I),
+    "lite_mask_geometry": ([_I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)], _I),
+    "lite_get_device_status": ([_P], _I),
+    "lite_status_string": ([_I], ctypes.c_char_p),
+    "lite_set_option": ([_I, ctypes.c_longlong], _I),
+    "lite_set_kernel_events": ([_P, _P], _I),
+}
+
+_lib = None
+
+
+class LiteAttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status} ({status_string(status)})")
+
+
+def load(path: str = LIB_PATH):
+    """Load the CUDA library (once). Raises if it is absent: there is no CPU path."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(f"CUDA library {path} is missing; build it with __graft_entry__.build()")
+        lib = ctypes.CDLL(path)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().lite_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != LITE_OK:
+        raise LiteAttnError(fn, status)
+
+
+def _stream_handle(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def lite_mask_geometry(N: int, d: int) -> Tuple[int, int, int]:
+    """(tile, T, W) for sequence length N and head dim d."""
+    tile, T, W = _I(), _I(), _I()
+    _check("lite_mask_geometry", load().lite_mask_geometry(int(N), int(d), ctypes.byref(tile), ctypes.byref(T),
+                                                           ctypes.byref(W)))
+    return tile.value, T.value, W.value
+
+
+def _check_qkv(q, k, v):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous 4-D bf16 CUDA tensor [B, N, H, d]")
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k, v must have the same shape [B, N, H, d]")
+
+
+def new_mask(B: int, H: int, N: int, d: int, device=None) -> torch.Tensor:
+    """A fresh (all-live) Skip-Mask, int32 [B, H, T, W] holding uint32 bit patterns."""
+    _, T, W = lite_mask_geometry(N, d)
+    return torch.zeros((B, H, T, W), dtype=torch.int32, device=device or "cuda")
+
+
+def lite_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask_in: Optional[torch.Tensor] = None,
+                  mask_out: Optional[torch.Tensor] = None, scale: Optional[float] = None, tau: float = -10.0,
+                  o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, return_lse: bool = True,
+                  stream=None):
+    """One LiteAttention forward (see include/lite_attn.h). Returns (o, lse or None)."""
+    _check_qkv(q, k, v)
+    B, N, H, d = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    for m in (mask_in, mask_out):
+        if m is not None and (m.dtype != torch.int32 or not m.is_contiguous() or not m.is_cuda):
+            raise ValueError("masks must be contiguous int32 CUDA tensors [B, H, T, W]")
+    st = load().lite_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _ptr(lse), _ptr(mask_in),
+                              _ptr(mask_out), B, H, N, d, float(scale or 0.0), float(tau), _stream_handle(stream))
+    _check("lite_attn_fwd", st)
+    return o, lse
+
+
+def lite_attn_dense(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float] = None,
+                    o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, return_lse: bool = True,
+                    stream=None):
+    """No-skip forward through the same kernel. Returns (o, lse or None)."""
+    _check_qkv(q, k, v)
+    B, N, H, d = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    st = load().lite_attn_dense(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _ptr(lse), B, H, N, d,
+                                float(scale or 0.0), _stream_handle(stream))
+    _check("lite_attn_dense", st)
+    return o, lse
+
+
+def lite_mask_to_list(mask: Optional[torch.Tensor], B: int, H: int, N: int, d: int, stream=None):
+    """Skip-Mask -> (list int16 [B,H,T,T], counts int32 [B,H,T]); list entries past counts are -1."""
+    _, T, W = lite_mask_geometry(N, d)
+    dev = mask.device if mask is not None else torch.device("cuda")
+    lst = torch.full((B, H, T, T), -1, dtype=torch.int16, device=dev)
+    counts = torch.empty((B, H, T), dtype=torch.int32, device=dev)
+    st = load().lite_mask_to_list(_ptr(mask), lst.data_ptr(), counts.data_ptr(), B, H, N, d, _stream_handle(stream))
+    _check("lite_mask_to_list", st)
+    return lst, counts
+
+
+def lite_schedule(counts: torch.Tensor, stream=None) -> torch.Tensor:
+    """Work order int32 [B*H*T] from live counts [B, H, T]."""
+    if counts.dtype != torch.int32 or not counts.is_contiguous() or counts.dim() != 3:
+        raise ValueError("counts must be contiguous int32 [B, H, T]")
+    B, H, T = counts.shape
+    order = torch.empty(B * H * T, dtype=torch.int32, device=counts.device)
+    _check("lite_schedule", load().lite_schedule(counts.data_ptr(), order.data_ptr(), B, H, T, _stream_handle(stream)))
+    return order
+
+
+def lite_get_device_status(stream=None) -> int:
+    """Synchronise and read/clear the device status word (0 = ok)."""
+    return load().lite_get_device_status(_stream_handle(stream))
+
+
+def lite_set_option(option: int, value: int):
+    _check("lite_set_option", load().lite_set_option(int(option), int(value)))
+
+
+def lite_set_kernel_events(before: Optional[torch.cuda.Event], after: Optional[torch.cuda.Event]):
+    """Record `before`/`after` around the attention kernel of later calls (None, None to stop)."""
+    b = before.cuda_event if before is not None else None
+    a = after.cuda_event if after is not None else None
+    _check("lite_set_kernel_events", load().lite_set_kernel_events(b, a))
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)
