@@ -1,0 +1,494 @@
+"""LiteAttention forward benchmark (one JSON line on rank 0).
+
+A step is one lite_attn_fwd call -- Skip-Mask compaction, LPT schedule and the block-sparse attention
+kernel with the fused QK-Skip test -- over one denoising step of a synthetic layer whose q, k, v are
+resident in HBM. The default workload is the 480p-like layer (B=1, H=40, N=32760 = 21x30x52, d=128,
+tile 128) over its 10-step trajectory with tau rising linearly from -10 to 0; steps past the
+trajectory keep tau at its last value. Every step reads fresh q/k/v (1.34 GB > L2), so no L2 flush
+is needed between timed steps.
+
+Reported: dense-equivalent TFLOP/s (4*B*H*N^2*d per step over the timed wall time) as `value`,
+executed TFLOP/s over the live tiles, the roofline of the attention kernel against the measured
+bf16 tensor peak, speedup against the dense path on the same inputs, an end-to-end number through
+host buffers, and the CPU oracle on a bounded sample.
+
+Multi-GPU (torchrun): each rank runs an independent layer of the same shape (its own seed): weak
+scaling with no data-path collective; only the timing scalar is reduced (max over ranks).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from temporal_block_sparse_b200 import workload as wlmod  # noqa: E402
+
+METRIC = "executed & dense-equiv attention TFLOP/s, % bf16 roofline, speedup vs dense at sparsity"
+KERNEL_SOURCES = ["temporal_block_sparse_b200/csrc/attn_kernel.cuh", "temporal_block_sparse_b200/csrc/sm100_ptx.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "lite_attn_kernel_480p_traffic.txt")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=7)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["lite", "reference"], default="lite")
+    ap.add_argument("--workload", default="480p", choices=sorted(wlmod.WORKLOADS))
+    ap.add_argument("--tau", type=float, default=None, help="fixed tau instead of the workload's schedule")
+    ap.add_argument("--cpu-sample-tiles", type=int, default=24, help="query tiles per step (reference arm)")
+    ap.add_argument("--heads", type=int, default=None, help="override H (a smaller layer, e.g. for profiling)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------------------- helpers
+
+
+def kernel_sha() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("bf16_tflops"), d.get("bf16_tflops_sustained"), "measured"
+    return 1590.0, 1400.0, "fallback"
+
+
+def stored_traffic(workload: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken on this kernel source."""
+    if workload != "480p" or not os.path.exists(TRAFFIC_FILE):
+        return None, None
+    txt = open(TRAFFIC_FILE).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    s = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
+    if not m or not s or s.group(1) != kernel_sha():
+        return None, None
+    return float(m.group(1)), txt
+
+
+def tau_at(wl, t, fixed):
+    if fixed is not None:
+        return fixed
+    return wl.tau(min(t, wl.steps - 1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling in the background (read-only queries)."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,utilization.gpu,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        rows = []
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        loaded = [r for r in rows if r[2] >= 50] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in loaded),
+                "reasons": reasons, "samples": len(loaded)}
+
+
+def live_flop(mask: torch.Tensor, N: int, d: int, tile: int) -> float:
+    """Executed FLOP of one step from its mask_in: sum over live (i, j) of 4 * rows_i * cols_j * d."""
+    B, H, T, W = mask.shape
+    words = mask.to(torch.int64) & 0xFFFFFFFF
+    shifts = torch.arange(32, device=mask.device, dtype=torch.int64)
+    bits = ((words.unsqueeze(-1) >> shifts) & 1).reshape(B, H, T, W * 32)[..., :T]
+    size = torch.full((T,), float(tile), device=mask.device, dtype=torch.float64)
+    size[T - 1] = N - (T - 1) * tile
+    live = 1.0 - bits.to(torch.float64)
+    return float(4.0 * d * torch.einsum("bhij,i,j->", live, size, size).item())
+
+
+def skipped_fraction(mask: torch.Tensor, T: int) -> float:
+    words = mask.to(torch.int64) & 0xFFFFFFFF
+    shifts = torch.arange(32, device=mask.device, dtype=torch.int64)
+    bits = ((words.unsqueeze(-1) >> shifts) & 1).reshape(*mask.shape[:3], -1)[..., :T]
+    return float(bits.to(torch.float64).mean().item())
+
+
+# ------------------------------------------------------------------------------------- CPU oracle
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def cpu_oracle_sample(q, k, v, mask_in, tau, budget_s=12.0, seed=0):
+    """Time the oracle on query tiles of one head (host copies of the GPU inputs), tile by tile,
+    until about `budget_s` seconds of CPU work have been spent (first and last tile always included)."""
+    import numpy as np
+
+    import oracle
+
+    B, N, H, d = q.shape
+    tile, T, _ = oracle.geometry(N, d)
+    rng = np.random.default_rng(seed)
+    b, h = 0, int(rng.integers(H))
+    order = [0, T - 1] + [int(x) for x in rng.permutation(np.arange(1, T - 1))]
+    sub = lambda x: x[b:b + 1, :, h:h + 1, :].float().cpu().numpy().astype(np.float64)
+    qs, ks, vs = sub(q), sub(k), sub(v)
+    m = mask_in[b:b + 1, h:h + 1].cpu().numpy().view(np.uint32)
+    spent, rows, done = 0.0, 0, 0
+    for i in order:
+        t0 = time.perf_counter()
+        oracle.lite_attention_forward(qs, ks, vs, m, tau=tau, query_tiles=[(0, 0, i)])
+        spent += time.perf_counter() - t0
+        rows += min(N, (i + 1) * tile) - i * tile
+        done += 1
+        if spent >= budget_s:
+            break
+    return 4.0 * rows * N * d, spent, f"{done} query tiles (b=0, h={h}) of one step, full key range"
+
+
+def run_reference(args):
+    """The oracle as it stands, on the host cores, with this benchmark's metric and workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+
+    wl = wlmod.WORKLOADS[args.workload]
+    # a bounded sample of the workload: one head's layer (B=1, H=1) drawn by the same recipe
+    sample_wl = wlmod.Workload(wl.name + "-1head", 1, 1, wl.frames, wl.grid_h, wl.grid_w, wl.d, wl.steps,
+                               wl.locality if wl.locality_range is None else sum(wl.locality_range) / 2,
+                               wl.drift, wl.tau_schedule, seed_offset=wl.seed_offset)
+    tr = wlmod.Trajectory(sample_wl, device="cpu")
+    N, d = wl.N, wl.d
+    _, T, W = oracle.geometry(N, d)
+    rng = np.random.default_rng(0)
+    tiles = sorted({0, T - 1} | {int(x) for x in rng.integers(0, T, size=max(args.cpu_sample_tiles - 2, 0))})
+    mask = np.zeros((1, 1, T, W), np.uint32)
+    times, flops = [], []
+    for t in range(args.warmup + args.steps):
+        q, k, v = (x.float().numpy().astype(np.float64) for x in tr.current())
+        t0 = time.perf_counter()
+        r = oracle.lite_attention_forward(q, k, v, mask, tau=tau_at(wl, t, args.tau),
+                                          query_tiles=[(0, 0, i) for i in tiles])
+        dt = time.perf_counter() - t0
+        mask = r.mask_out
+        tl = oracle.tile_for_head_dim(d)
+        rows = sum(min(N, (i + 1) * tl) - i * tl for i in tiles)
+        if t >= args.warmup:
+            times.append(dt)
+            flops.append(4.0 * rows * N * d)
+        tr.advance()
+    value = sum(flops) / sum(times) / 1e12
+    cores = oracle_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{wl.name} layer", "B": wl.B, "H": wl.H, "N": N, "d": d,
+                   "sample": f"{len(tiles)} query tiles of one head per step"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{len(tiles)} query tiles x full key range of one head, per step; "
+                                   f"dense-equivalent FLOP"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------- GPU arm
+
+
+def rank_workload(base, rank: int, heads=None):
+    """Rank r's problem: an independent layer of the base shape with its own seed (weak scaling)."""
+    return wlmod.Workload(base.name, base.B, heads or base.H, base.frames, base.grid_h, base.grid_w, base.d,
+                          base.steps, base.locality, base.drift, base.tau_schedule, base.locality_range,
+                          seed_offset=base.seed_offset + 1000 * rank)
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """Slowest rank's time (the only collective of the benchmark)."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    from temporal_block_sparse_b200 import lite_attn as la
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    la.load()
+
+    wl = rank_workload(wlmod.WORKLOADS[args.workload], rank, args.heads)
+    B, N, H, d = wl.B, wl.N, wl.H, wl.d
+    tile, T, W = la.lite_mask_geometry(N, d)
+    S = args.warmup + args.steps
+
+    # inputs of every step, resident in HBM before timing
+    tr = wlmod.Trajectory(wl, device=dev)
+    qkv = []
+    for t in range(S):
+        qkv.append(tr.current())
+        tr.advance()
+    del tr
+    masks = [torch.zeros((B, H, T, W), dtype=torch.int32, device=dev) for _ in range(S + 1)]
+    o = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def fwd(t, out=o, out_lse=lse):
+        q, k, v = qkv[t]
+        la.lite_attn_fwd(q, k, v, masks[t], masks[t + 1], tau=tau_at(wl, t, args.tau), o=out, lse=out_lse)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    for t in range(args.warmup):
+        fwd(t)
+    torch.cuda.synchronize()
+    assert la.lite_get_device_status() == 0
+
+    # ---- timed region: exactly K steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in ev:  # create the events before handing them to the library
+        a.record()
+        b.record()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(args.steps):
+        la.lite_set_kernel_events(*ev[i])
+        fwd(args.warmup + i)
+    end.record()
+    la.lite_set_kernel_events(None, None)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clock_info = clocks.stop()
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), dist, dev)
+    status = la.lite_get_device_status()
+    assert status == 0, la.status_string(status)
+    attn_ms = [a.elapsed_time(b) for a, b in ev]
+
+    timed = range(args.warmup, S)
+    dense_flop_step = wl.dense_flop()
+    exec_flop = [live_flop(masks[t], N, d, tile) for t in timed]
+    skip_frac = [skipped_fraction(masks[t], T) for t in timed]
+    total_dense = dense_flop_step * args.steps * world
+    value = total_dense / (elapsed_ms * 1e-3) / 1e12
+    executed_tflops = sum(exec_flop) * world / (elapsed_ms * 1e-3) / 1e12
+
+    # ---- dense path on the same inputs (context for the speedup; not part of the step)
+    d_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in timed]
+    for i, t in enumerate(timed):
+        q, k, v = qkv[t]
+        d_ev[i][0].record()
+        la.lite_attn_dense(q, k, v, o=o, lse=lse)
+        d_ev[i][1].record()
+    torch.cuda.synchronize()
+    dense_ms = sum(a.elapsed_time(b) for a, b in d_ev)
+    sparse_ms = elapsed_ms
+
+    # ---- roofline of the attention kernel (executed FLOP per launch / its event-timed duration)
+    burst, sustained, peak_src = measured_peaks()
+    attn_avg_ms = sum(attn_ms) / len(attn_ms)
+    flop_per_launch = sum(exec_flop) / len(exec_flop)
+    achieved = flop_per_launch / (attn_avg_ms * 1e-3) / 1e12
+    traffic, _ = stored_traffic(args.workload)
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                "frac": achieved / burst, "traffic": traffic,
+                "peak_kind": f"{peak_src} bf16 dense burst (cuBLAS); sustained {sustained}",
+                "frac_of_sustained": achieved / sustained, "kernel": "lite_attn_kernel<128,128>",
+                "attn_ms_per_launch": attn_avg_ms, "attn_share_of_step": sum(attn_ms) / elapsed_ms}
+
+    # ---- end to end through host buffers (pinned), copies overlapped with compute
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, la, wl, qkv, masks, dev, world, dist)
+
+    # ---- CPU oracle on a bounded sample (rank 0, N=1 only)
+    cpu = None
+    if not args.no_cpu and world == 1 and rank == 0:
+        t_mid = args.warmup + args.steps // 2
+        q, k, v = qkv[t_mid]
+        fl, dt, what = cpu_oracle_sample(q, k, v, masks[t_mid], tau_at(wl, t_mid, args.tau))
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+               "sample": f"{what}; dense-equivalent FLOP / oracle wall time ({dt:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{wl.name} layer: B={B} H={H} N={N} ({wl.frames}x{wl.grid_h}x{wl.grid_w}) "
+                                   f"d={d} tile={tile}, denoising steps {args.warmup}..{S - 1} of the trajectory",
+                       "B": B, "H": H, "N": N, "d": d, "tile": tile,
+                       "tau": [tau_at(wl, t, args.tau) for t in timed],
+                       "global_batch": B * world, "parallelism": f"dp{world}",
+                       "l2": "inputs larger than L2: fresh 1.34+ GB q/k/v every step, no flush needed"},
+            "executed_tflops": executed_tflops,
+            "dense_equiv_tflops": value,
+            "skipped_tile_fraction": skip_frac,
+            "speedup_vs_dense": dense_ms / sparse_ms,
+            "dense_path_tflops": total_dense / world / (dense_ms * 1e-3) / 1e12,
+            "roofline": roofline,
+            "gpu_launches": 3 * args.steps,
+            "clocks": clock_info,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(args, la, wl, qkv, masks, dev, world, dist):
+    """Same K steps through host buffers: H2D of q/k/v and D2H of o/lse inside the timed region.
+
+    Copies run on a side stream, double buffered, so step t+1's inputs upload while step t computes.
+    """
+    B, N, H, d = wl.B, wl.N, wl.H, wl.d
+    timed = list(range(args.warmup, args.warmup + args.steps))
+    host_in = []
+    for t in timed:
+        bufs = tuple(torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in qkv[t])
+        for hb, x in zip(bufs, qkv[t]):
+            hb.copy_(x)
+        host_in.append(bufs)
+    host_o = [torch.empty((B, N, H, d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    host_l = [torch.empty((B, H, N), dtype=torch.float32).pin_memory() for _ in range(2)]
+    dev_in = [tuple(torch.empty_like(x) for x in qkv[0]) for _ in range(2)]
+    dev_o = [torch.empty((B, N, H, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    dev_l = [torch.empty((B, H, N), dtype=torch.float32, device=dev) for _ in range(2)]
+    e_masks = [m.clone() for m in masks]
+    comp = torch.cuda.current_stream()
+    copy = torch.cuda.Stream()
+    up_done = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    down_done = [torch.cuda.Event() for _ in range(2)]
+    h2d = sum(x.numel() * x.element_size() for x in host_in[0])
+    d2h = host_o[0].numel() * 2 + host_l[0].numel() * 4
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(comp)
+
+    def upload(i):
+        s = i % 2
+        with torch.cuda.stream(copy):
+            if i >= 2:
+                copy.wait_event(comp_done[s])  # slot free once step i-2 has computed
+            for dst, src in zip(dev_in[s], host_in[i]):
+                dst.copy_(src, non_blocking=True)
+            up_done[s].record(copy)
+
+    upload(0)
+    for i, t in enumerate(timed):
+        s = i % 2
+        if i + 1 < len(timed):
+            upload(i + 1)
+        comp.wait_event(up_done[s])
+        if i >= 2:
+            comp.wait_event(down_done[s])  # output slot read back
+        q, k, v = dev_in[s]
+        la.lite_attn_fwd(q, k, v, e_masks[t], e_masks[t + 1], tau=tau_at(wl, t, args.tau), o=dev_o[s], lse=dev_l[s])
+        comp_done[s].record(comp)
+        with torch.cuda.stream(copy):
+            copy.wait_event(comp_done[s])
+            host_o[s].copy_(dev_o[s], non_blocking=True)
+            host_l[s].copy_(dev_l[s], non_blocking=True)
+            down_done[s].record(copy)
+    comp.wait_stream(copy)
+    end.record(comp)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(start.elapsed_time(end), dist, dev)
+    value = wl.dense_flop() * len(timed) * world / (ms * 1e-3) / 1e12
+    return {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": ms / len(timed), "note": "pinned host q/k/v in, o/lse out; copies overlap compute"}
+
+
+if __name__ == "__main__":
+    main()
