@@ -46,7 +46,8 @@ enum {
   LITE_ERR_UNSUPPORTED = -2, /* d not in {64, 128}, misaligned pointer, T or sizes beyond limits  */
   LITE_ERR_CUDA = -3,        /* a CUDA launch, allocation or query failed                          */
   LITE_ERR_TIMEOUT = -4,     /* device status: a kernel wait exceeded its time limit and gave up   */
-  LITE_ERR_CHECK = -5        /* device status: an in-kernel consistency check failed               */
+  LITE_ERR_CHECK = -5,       /* device status: an in-kernel consistency check failed               */
+  LITE_ERR_SCRATCH_LIMIT = -6 /* lite_attn_fwd_noalloc: the layer needs more than its fixed scratch  */
 };
 
 /*
@@ -154,6 +155,38 @@ int lite_set_option(int option, long long value);
  * the call's stream. Both are cudaEvent_t handles owned by the caller; pass NULL, NULL to stop.
  */
 int lite_set_kernel_events(void* before, void* after);
+
+/*
+ * lite_attn_fwd_noalloc -- lite_attn_fwd for callers that must not allocate device memory.
+ *
+ * The LiteAttention paper and pages have no counterpart to this entry point; it exists for
+ * embedding the forward pass where the library may not allocate: a serving runtime that has
+ * reserved (nearly) all device memory for its own pool, so any allocation by a library fails or
+ * evicts the caller's data, or a latency-critical denoising loop that cannot afford an
+ * allocator call (which may block or synchronise) on every layer of every step.
+ *
+ * Arguments, layouts, semantics and results are exactly those of lite_attn_fwd. The difference is
+ * where the per-call scratch (live lists, counts, work order, work counter) lives: in one fixed
+ * array of LITE_NOALLOC_SCRATCH_BYTES (8 MiB) that the library defines in device memory. Every GPU
+ * that loads the library holds that array until the process exits. This call makes no cudaMalloc,
+ * cudaFree or other allocating call.
+ *
+ *  - Limit: the layer's scratch must fit in 8 MiB. With R = B*H*T and T = ceil(N / tile) it is
+ *    up256(2*R*T) + 2*up256(4*R) + 256 bytes (up256 rounds up to a multiple of 256), about
+ *    R*(2T + 8). The 480p layer (B=1, H=40, N=32760, d=128: 5.3 MB) fits; the 720p layer
+ *    (N=75600: 28 MB) does not. Layers that do not fit return LITE_ERR_SCRATCH_LIMIT before any
+ *    work is enqueued.
+ *  - Set-up: the first call on each device looks up the array's device address (with that device
+ *    current); make that first call before capturing any stream into a CUDA graph.
+ *  - Sharing: all calls on a device use the same array, and it keeps whatever the last call left
+ *    in it (the work counter is cleared on the stream at the start of every call). Calls whose
+ *    work overlaps on the GPU -- for example on two streams without ordering between them --
+ *    race on the array and give wrong results; order them on one stream or with events.
+ */
+#define LITE_NOALLOC_SCRATCH_BYTES (8u << 20)
+int lite_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                          const uint32_t* mask_in, uint32_t* mask_out, int B, int H, int N, int d,
+                          float scale, float tau, lite_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -187,6 +187,7 @@ const char* lite_status_string(int status) {
     case LITE_ERR_CUDA: return "CUDA launch, allocation or query failed";
     case LITE_ERR_TIMEOUT: return "a kernel wait exceeded its time limit; outputs of that call are invalid";
     case LITE_ERR_CHECK: return "an in-kernel consistency check failed";
+    case LITE_ERR_SCRATCH_LIMIT: return "layer needs more scratch than lite_attn_fwd_noalloc's fixed 8 MiB";
     default: return "unknown status";
   }
 }
@@ -324,3 +325,82 @@ int lite_attn_dense(const void* q, const void* k, const void* v, void* o, float*
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// No-allocation variant of lite_attn_fwd.
+//
+// Its scratch lives in the file-scope device array below, which every device holds once the
+// library is loaded on it. In host code `g_noalloc_scratch` is only a host-side stand-in for the
+// symbol, not a device address: its device address is looked up once per device with
+// cudaGetSymbolAddress (device current) and that address is what the kernels receive.
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LITE_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_addr[kMaxDevices] = {nullptr};
+
+// First call on a device: find the array's device address. Returns nullptr on failure.
+void* noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return nullptr;
+    g_noalloc_addr[dev] = ptr;
+  }
+  return g_noalloc_addr[dev];
+}
+
+}  // namespace
+
+extern "C" int lite_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                                     const uint32_t* mask_in, uint32_t* mask_out, int B, int H, int N, int d,
+                                     float scale, float tau, lite_stream_t stream) {
+  int st = check_qkvo(q, k, v, o, lse);
+  if (st) return st;
+  st = check_shapes(B, H, N, d);
+  if (st) return st;
+  if (std::isnan(tau)) return LITE_ERR_INVALID_ARG;
+  if (tau > 0.f && !debug_env()) return LITE_ERR_INVALID_ARG;
+  if ((mask_in && (reinterpret_cast<uintptr_t>(mask_in) & 3u)) || (mask_out && (reinterpret_cast<uintptr_t>(mask_out) & 3u)))
+    return LITE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > 8192) return LITE_ERR_UNSUPPORTED;
+
+  const int t = tile_for(d);
+  const int T = (N + t - 1) / t;
+  const size_t rows = size_t(B) * H * T;
+  const size_t list_b = align256(rows * T * sizeof(int16_t));
+  const size_t cnt_b = align256(rows * sizeof(int32_t));
+  const size_t need = list_b + 2 * cnt_b + 256;
+  if (need > LITE_NOALLOC_SCRATCH_BYTES) return LITE_ERR_SCRATCH_LIMIT;
+
+  DeviceCache* dc = nullptr;
+  if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
+  char* base = static_cast<char*>(noalloc_scratch());
+  if (!base) return LITE_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  lite::AttnParams p = base_params(o, lse, B, H, N, d, scale, dc);
+  const int W = p.W;
+  int16_t* list = reinterpret_cast<int16_t*>(base);
+  int32_t* counts = reinterpret_cast<int32_t*>(base + list_b);
+  int32_t* order = reinterpret_cast<int32_t*>(base + list_b + cnt_b);
+  int32_t* counter = reinterpret_cast<int32_t*>(base + list_b + 2 * cnt_b);
+
+  // the array keeps the previous call's contents: the work counter must start at zero
+  if (cudaMemsetAsync(counter, 0, sizeof(int32_t), s) != cudaSuccess) return LITE_ERR_CUDA;
+  lite::lite_compact_kernel<<<(int(rows) + 7) / 8, 256, 0, s>>>(mask_in, mask_out, list, counts, int(rows), T, W);
+  if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
+  const size_t sm = size_t(B * H + T) * sizeof(int32_t);
+  lite::lite_schedule_kernel<<<B * H, 512, sm, s>>>(counts, order, B * H, T);
+  if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
+  p.mask_out = mask_out;
+  p.list = list;
+  p.counts = counts;
+  p.order = order;
+  p.work_counter = counter;
+  p.tau_log2 = tau * 1.4426950408889634f;
+  p.skip_test = (mask_out != nullptr && tau > -INFINITY) ? 1 : 0;
+  return run_attention(dc, d, q, k, v, p, s);
+}

@@ -23,6 +23,8 @@ LITE_ERR_UNSUPPORTED = -2
 LITE_ERR_CUDA = -3
 LITE_ERR_TIMEOUT = -4
 LITE_ERR_CHECK = -5
+LITE_ERR_SCRATCH_LIMIT = -6
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 LITE_OPT_WAIT_LIMIT_NS = 1
 LITE_OPT_DEBUG_STALL = 2
@@ -42,6 +44,7 @@ SIGNATURES = {
     "lite_status_string": ([_I], ctypes.c_char_p),
     "lite_set_option": ([_I, ctypes.c_longlong], _I),
     "lite_set_kernel_events": ([_P, _P], _I),
+    "lite_attn_fwd_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _F, _P], _I),
 }
 
 _lib = None
@@ -184,3 +187,22 @@ def lite_set_kernel_events(before: Optional[torch.cuda.Event], after: Optional[t
 
 def default_scale(d: int) -> float:
     return 1.0 / math.sqrt(d)
+
+
+def lite_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                          lse: Optional[torch.Tensor] = None, mask_in: Optional[torch.Tensor] = None,
+                          mask_out: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+                          tau: float = -10.0, stream=None):
+    """lite_attn_fwd for callers that must not allocate device memory (see include/lite_attn.h).
+
+    The library allocates nothing here: the caller passes every output buffer, and the per-call
+    scratch sits in the library's fixed 8 MiB device array (layers needing more are refused with
+    LITE_ERR_SCRATCH_LIMIT). Calls that overlap on the GPU race on that array.
+    """
+    _check_qkv(q, k, v)
+    B, N, H, d = q.shape
+    st = load().lite_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _ptr(lse),
+                                      _ptr(mask_in), _ptr(mask_out), B, H, N, d, float(scale or 0.0), float(tau),
+                                      _stream_handle(stream))
+    _check("lite_attn_fwd_noalloc", st)
+    return o, lse
