@@ -5,16 +5,24 @@
 // Elimination": a skipped tile costs no K/V load, no QK^T, no softmax, no PV), from the highest
 // key-tile index down (README, must_do_list: "we iterate in reverse order inside of the kernel").
 //
-// Warp roles (192 threads):
-//   warp 0       TMA producer: Q once per item, then K_j and V_j per live tile into a 2-stage ring.
-//   warp 1       TMEM allocator and single-thread tcgen05 MMA issuer:
-//                  S_j = Q K_j^T  (SS form, fp32 accumulators in TMEM, double buffered),
-//                  O  += P_j V_j  (TS form: P read from TMEM, V from shared memory).
-//   warps 2..5   softmax: one thread per query row (TMEM lane). Per tile: row max, the QK-Skip
-//                vote (skill page "Lite Attention Temporal Sparse", Core Concept: a tile whose local
-//                max score is far below the cumulative max is flagged), one atomicOr per flagged
-//                (query tile, key tile), exp2, row sum, P (bf16) back to TMEM, O rescale when the
-//                running max moved by more than 2^8; epilogue O / l and lse.
+// Warp roles (320 threads):
+//   warp 0       TMA producer: Q once per item; per live tile K_j into a 2-stage ring and V_j into
+//                a 3-stage ring (separate barriers, so S = QK^T never waits for V).
+//   warp 1       TMEM allocator and single-thread tcgen05 MMA issuer, in the order
+//                QK_0, QK_1, PV_0, QK_2, PV_1, ... over the live tiles of consecutive items:
+//                  S_t = Q K_t^T  (SS form) into TMEM buffer t%2,
+//                  O_{t%2} += P_t V_t (TS form: P read from TMEM, V from shared memory).
+//   warps 2..5   softmax warpgroup 0: the tiles t with t%2 == 0;  warps 6..9: warpgroup 1, t%2 == 1.
+//                One thread per query row (TMEM lane). The two groups work on consecutive tiles at
+//                the same time, each with its own running exponent reference, row sum and O
+//                accumulator; the epilogue combines the two partial softmaxes exactly. Per tile:
+//                row max; the QK-Skip vote (skill page "Lite Attention Temporal Sparse", Core
+//                Concept: a tile whose local max score is far below the cumulative max is
+//                flagged) against the running max over ALL earlier tiles, for which each group
+//                receives the other's tile maxima through a shared-memory mailbox; one atomicOr
+//                per flagged (query tile, key tile); exp2 (a quarter on the FMA pipe); P (bf16)
+//                back into TMEM over the consumed S columns; O rescale when the group's reference
+//                max grew by more than 2^8.
 //
 // Every wait is bounded by a wall-clock limit; on expiry the kernel records a timeout in the device
 // status word, every role stops, in-flight copies and MMAs are drained, TMEM is freed and the CTA
@@ -46,32 +54,52 @@ struct AttnParams {
   int skip_test;            // 1: run the QK-Skip vote and record flags
   unsigned long long wait_limit_ns;
   int debug_stall;          // test hook: MMA warp withholds its first tile
+#ifdef LITE_ATTN_TRACE
+  long long* trace;         // [4 CTAs][4 roles][8 events][512 tiles] clock64 stamps
+#endif
 };
+
+// Timing probes for analysis builds (-DLITE_ATTN_TRACE); empty in the library build.
+#ifdef LITE_ATTN_TRACE
+#define LITE_TRACE(role, ev, t)                                                                        \
+  do {                                                                                                 \
+    if (p.trace && blockIdx.x < 4 && uint32_t(t) < 512u)                                               \
+      p.trace[(((blockIdx.x * 4 + (role)) * 8 + (ev)) * 512) + uint32_t(t)] = clock64();               \
+  } while (0)
+#else
+#define LITE_TRACE(role, ev, t) \
+  do {                          \
+  } while (0)
+#endif
 
 template <int D, int BN>
 struct AttnCfg {
   static constexpr int BM = 128;                 // MMA M = TMEM lanes = query rows of the tile slot
   static constexpr int BQ = BN;                  // valid query rows per query tile
-  static constexpr int STAGES = 2;               // K/V ring depth
+  static constexpr int KST = 2;                  // K stages
+  static constexpr int VST = 3;                  // V stages
+  static constexpr int THREADS = 320;            // producer warp, MMA warp, 2 softmax warpgroups
   static constexpr int NCHUNK = D / 64;          // 128-byte swizzle atoms along d
   static constexpr int Q_CHUNK = BM * 128;       // bytes between d-chunks of Q in smem
   static constexpr int KV_CHUNK = BN * 128;      // bytes between d-chunks of a K or V tile
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr uint32_t Q_TX = BQ * D * 2;   // bytes the Q load delivers
-  static constexpr uint32_t KV_TX = BN * D * 2;
+  static constexpr uint32_t KV_TX = BN * D * 2;  // bytes of one K or V tile
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-  static constexpr int OFF_CTL = OFF_V + STAGES * KV_BYTES;
+  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
+  static constexpr int OFF_CTL = OFF_V + VST * KV_BYTES;
   static constexpr int CTL_BYTES = 512;
+  static constexpr int OFF_X = OFF_CTL + CTL_BYTES;  // tile-max mailbox float[4][128]; epilogue float[2][2][128]
+  static constexpr int X_BYTES = 4 * 128 * 4 + 2 * 2 * 128 * 4;
   // one CTA per SM: the request is padded so that two never fit (TMEM is sized for one)
-  static constexpr int SMEM_USED = OFF_CTL + CTL_BYTES + 1024;
+  static constexpr int SMEM_USED = OFF_X + X_BYTES + 1024;
   static constexpr int SMEM_BYTES = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
-  // TMEM columns: S buffers at [0, BN) and [BN, 2BN); O at [2BN, 2BN + D)
+  // TMEM columns: S_0 [0, BN), S_1 [BN, 2BN), O_0 [2BN, 2BN+D), O_1 [2BN+D, 2BN+2D)
   static constexpr uint32_t S_COL = 0;
   static constexpr uint32_t O_COL = 2 * BN;
-  static constexpr uint32_t TMEM_COLS = (2 * BN + D) <= 256 ? 256 : 512;
+  static constexpr uint32_t TMEM_COLS = (2 * BN + 2 * D) <= 256 ? 256 : 512;
   // instruction descriptors, kind::f16: fp32 accumulate (bit 4), bf16 A (bits 7-9) and B (10-12),
   // B major-ness (bit 16), N >> 3 (bits 17-22), M >> 4 (bits 24-28)
   static constexpr uint32_t IDESC_QK = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) |
@@ -80,15 +108,18 @@ struct AttnCfg {
                                        (uint32_t(D >> 3) << 17) | (uint32_t(BM >> 4) << 24);
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(BN == 64 || BN == 128, "tile");
-  static_assert(2 * BN + D <= 512, "TMEM budget");
+  static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 // Control block in shared memory (barriers are 8-byte mbarrier objects).
 struct alignas(8) AttnCtl {
   uint64_t q_full, q_empty;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t s_full[2], p_full[2];
-  uint64_t pv_done, o_free;
+  uint64_t k_full[2], v_full[3];     // K_t (stage t%2) / V_t (stage t%3) landed
+  uint64_t s_full[2], p_full[2];     // S_t ready / P_t written (buffer t%2, one warpgroup each)
+  uint64_t pv_done[2];               // last PV of group g in an item finished (accumulator g)
+  uint64_t mx_full[4];               // row maxima of tile t posted in mailbox slot t%4
+  uint64_t o_free;                   // epilogue has read both O accumulators
   uint64_t item_full[2], item_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
@@ -105,6 +136,37 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo
   d |= uint64_t(1) << 46;
   d |= uint64_t(2) << 61;
   return d;
+}
+
+// 2^x on the FMA/ALU pipes, for the share of the exponentials taken off the MUFU unit.
+// Range reduction in the manner of Cody and Waite: adding 1.5*2^23 rounds x to the nearest integer
+// n in the low mantissa bits of t, f = x - n lies in [-1/2, 1/2], 2^f comes from a cubic, and n is
+// added to the exponent field. The cubic interpolates 2^f at the four Chebyshev nodes of
+// [-1/2, 1/2] (max relative error 1.0e-4, far below the 2^-9 rounding of the bf16 P it feeds).
+// x is clamped at -126 so the exponent field stays valid; results below 2^-126 are immaterial here.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(0.05583828315138817f, f, 0.2426394820213318f), f, 0.6931367516517639f), f,
+                       0.9999245405197144f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// The same 2^x for two values with packed fp32x2 arithmetic (identical float32 steps, so identical
+// results): 12 instructions for two exponentials instead of two MUFU operations.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
+  float2 q = __ffma2_rn(make_float2(0.05583828315138817f, 0.05583828315138817f), f,
+                        make_float2(0.2426394820213318f, 0.2426394820213318f));
+  q = __ffma2_rn(q, f, make_float2(0.6931367516517639f, 0.6931367516517639f));
+  q = __ffma2_rn(q, f, make_float2(0.9999245405197144f, 0.9999245405197144f));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
 struct Waiter {
@@ -166,13 +228,16 @@ __device__ __forceinline__ int key_tile(const AttnParams& p, int row, int idx) {
 }
 
 template <int D, int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     lite_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using C = AttnCfg<D, BN>;
+  static_assert(sizeof(AttnCtl) <= C::CTL_BYTES, "control block");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   AttnCtl* ctl = reinterpret_cast<AttnCtl*>(smem + C::OFF_CTL);
+  float* mailbox = reinterpret_cast<float*>(smem + C::OFF_X);    // [4][128] tile row maxima
+  float* epi = mailbox + 4 * 128;                                // [2 groups][2 values][128]
   const uint32_t sQ = ptx::smem_addr(smem + C::OFF_Q);
   const uint32_t sK = ptx::smem_addr(smem + C::OFF_K);
   const uint32_t sV = ptx::smem_addr(smem + C::OFF_V);
@@ -184,18 +249,17 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     ptx::mbar_init(BAR(q_full), 1);
     ptx::mbar_init(BAR(q_empty), 1);
-    for (int s = 0; s < 2; ++s) {
-      ptx::mbar_init(BAR(k_full[s]), 1);
-      ptx::mbar_init(BAR(k_empty[s]), 1);
-      ptx::mbar_init(BAR(v_full[s]), 1);
-      ptx::mbar_init(BAR(v_empty[s]), 1);
-      ptx::mbar_init(BAR(s_full[s]), 1);
-      ptx::mbar_init(BAR(p_full[s]), 128);
-      ptx::mbar_init(BAR(item_full[s]), 1);
-      ptx::mbar_init(BAR(item_empty[s]), 5);  // MMA thread + one lane of each softmax warp
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(BAR(k_full[b]), 1);
+      ptx::mbar_init(BAR(s_full[b]), 1);
+      ptx::mbar_init(BAR(p_full[b]), 128);
+      ptx::mbar_init(BAR(pv_done[b]), 1);
+      ptx::mbar_init(BAR(item_full[b]), 1);
+      ptx::mbar_init(BAR(item_empty[b]), 9);  // MMA thread + one lane of each softmax warp
     }
-    ptx::mbar_init(BAR(pv_done), 1);
-    ptx::mbar_init(BAR(o_free), 128);
+    for (int b = 0; b < 3; ++b) ptx::mbar_init(BAR(v_full[b]), 1);
+    for (int b = 0; b < 4; ++b) ptx::mbar_init(BAR(mx_full[b]), 128);
+    ptx::mbar_init(BAR(o_free), 256);
     ptx::mbar_init(BAR(drain), 1);
     ctl->abort = 0;
     ptx::fence_mbar_init();
@@ -221,14 +285,19 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = ctl->tmem_base;
   const Waiter wt{&ctl->abort, p.status, p.wait_limit_ns};
 
+  // Barrier phases: t counts the live tiles of all items this CTA processes, in processing order.
+  // Tile t uses S buffer, P slot, accumulator and softmax warpgroup t%2, K stage t%2, V stage t%3,
+  // mailbox slot t%4. Every waiter either observes each phase of a barrier in order, or is
+  // guaranteed by the order of the MMA thread's commits that the barrier is at most one phase
+  // away from the awaited one, so the parity waits are exact.
   if (warp == 0) {
     // ------------------------------------------------------------------------- TMA producer
     if (lane == 0) {
-      uint32_t kv = 0, items = 0, qn = 0;
+      uint32_t t = 0, items = 0, qn = 0;
       bool ok = true;
       // last armed phase of each full barrier, so that every issued load can be drained at exit
-      bool q_armed = false, k_armed[2] = {false, false}, v_armed[2] = {false, false};
-      uint32_t q_par = 0, k_par[2] = {0, 0}, v_par[2] = {0, 0};
+      bool q_armed = false, k_armed[2] = {false, false}, v_armed[3] = {false, false, false};
+      uint32_t q_par = 0, k_par[2] = {0, 0}, v_par[3] = {0, 0, 0};
       while (ok) {
         const int slot = items & 1;
         if (items >= 2) ok = wt.wait(BAR(item_empty[slot]), ((items >> 1) - 1) & 1);
@@ -250,60 +319,57 @@ __global__ void __launch_bounds__(192, 1)
         q_armed = true;
         q_par = qn & 1;
         ++qn;
-        for (int idx = 0; idx < it.n && ok; ++idx, ++kv) {
+        for (int idx = 0; idx < it.n && ok; ++idx, ++t) {
           const int j = key_tile(p, it.row, idx);
-          const int s = kv & 1;
-          const uint32_t ph = (kv >> 1) & 1;
-          if (kv >= 2) ok = wt.wait(BAR(k_empty[s]), ph ^ 1);
+          // K stage t%2 is free once QK_{t-2} finished. V stage t%3 is free once PV_{t-3} finished,
+          // which is implied by QK_{t-1} finishing: the MMA thread issues PV_{t-3} before QK_{t-1}
+          // and a commit covers every earlier MMA. The s_full barrier of a buffer can only move past
+          // the awaited phase after a K load this thread has not issued yet, so the waits are exact.
+          LITE_TRACE(0, 0, t);
+          if (t >= 2) ok = wt.wait(BAR(s_full[t & 1]), ((t - 2) >> 1) & 1);
           if (!ok) break;
-          ptx::mbar_arrive_expect_tx(BAR(k_full[s]), C::KV_TX);
+          ptx::mbar_arrive_expect_tx(BAR(k_full[t & 1]), C::KV_TX);
           for (int c = 0; c < C::NCHUNK; ++c)
-            ptx::tma_load_4d(sK + s * C::KV_BYTES + c * C::KV_CHUNK, &tmK, BAR(k_full[s]), c * 64, it.h,
+            ptx::tma_load_4d(sK + (t & 1) * C::KV_BYTES + c * C::KV_CHUNK, &tmK, BAR(k_full[t & 1]), c * 64, it.h,
                              j * BN, it.b);
-          k_armed[s] = true;
-          k_par[s] = ph;
-          if (kv >= 2) ok = wt.wait(BAR(v_empty[s]), ph ^ 1);
+          LITE_TRACE(0, 1, t);
+          k_armed[t & 1] = true;
+          k_par[t & 1] = (t >> 1) & 1;
+          const uint32_t vs = t % 3;
+          if (t >= 3) ok = wt.wait(BAR(s_full[(t - 1) & 1]), ((t - 1) >> 1) & 1);
           if (!ok) break;
-          ptx::mbar_arrive_expect_tx(BAR(v_full[s]), C::KV_TX);
+          ptx::mbar_arrive_expect_tx(BAR(v_full[vs]), C::KV_TX);
           for (int c = 0; c < C::NCHUNK; ++c)
-            ptx::tma_load_4d(sV + s * C::KV_BYTES + c * C::KV_CHUNK, &tmV, BAR(v_full[s]), c * 64, it.h,
-                             j * BN, it.b);
-          v_armed[s] = true;
-          v_par[s] = ph;
+            ptx::tma_load_4d(sV + vs * C::KV_BYTES + c * C::KV_CHUNK, &tmV, BAR(v_full[vs]), c * 64, it.h, j * BN,
+                             it.b);
+          LITE_TRACE(0, 3, t);
+          v_armed[vs] = true;
+          v_par[vs] = (t / 3) & 1;
         }
       }
       // Drain: every issued TMA load has landed before this thread leaves (no other thread arms these
       // barriers, so the last armed phase is the one to wait for).
       if (q_armed) wt.wait_drain(BAR(q_full), q_par);
-      for (int s = 0; s < 2; ++s) {
-        if (k_armed[s]) wt.wait_drain(BAR(k_full[s]), k_par[s]);
-        if (v_armed[s]) wt.wait_drain(BAR(v_full[s]), v_par[s]);
-      }
+      for (int b = 0; b < 2; ++b)
+        if (k_armed[b]) wt.wait_drain(BAR(k_full[b]), k_par[b]);
+      for (int b = 0; b < 3; ++b)
+        if (v_armed[b]) wt.wait_drain(BAR(v_full[b]), v_par[b]);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------------- MMA issuer
+    // The tensor pipe only buffers about 100 cycles of issue gaps, so this loop is kept lean:
+    // descriptors are built once and advanced by 32-bit adds, and per tile there are three waits
+    // (K, P, V) and one commit.
     if (lane == 0) {
-      uint32_t kv = 0, g = 0, items = 0, qn = 0;
+      uint32_t t0 = 0, items = 0, qn = 0;
       bool ok = true;
       bool stalled = false;
-      auto issue_pv = [&](uint32_t gi, uint32_t kvi, bool first_of_item) -> bool {
-        const uint32_t buf = gi & 1;
-        const uint32_t s = kvi & 1;
-        if (!wt.wait(BAR(p_full[buf]), (gi >> 1) & 1)) return false;
-        if (!wt.wait(BAR(v_full[s]), (kvi >> 1) & 1)) return false;
-        ptx::tc_fence_after();
-        const uint32_t p_tmem = tmem + C::S_COL + buf * BN;
-        const uint32_t v_base = sV + s * C::KV_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bdesc = umma_desc_sw128(v_base + kk * 2048, C::KV_CHUNK, 1024);
-          ptx::mma_ts(tmem + C::O_COL, p_tmem + kk * 8, bdesc, C::IDESC_PV, (first_of_item && kk == 0) ? 0u : 1u);
-        }
-        ptx::mma_commit(BAR(pv_done));
-        ptx::mma_commit(BAR(v_empty[s]));
-        return true;
-      };
+      // 128B-swizzled K-major operands advance 32 bytes (>> 4 = 2) per K=16 step inside an atom;
+      // V (MN-major) advances 16 rows = 2048 bytes (>> 4 = 128) per step.
+      const uint64_t q_desc = umma_desc_sw128(sQ, 16, 1024);
+      const uint64_t k_desc0 = umma_desc_sw128(sK, 16, 1024);
+      const uint64_t v_desc0 = umma_desc_sw128(sV, C::KV_CHUNK, 1024);
       while (ok) {
         const int slot = items & 1;
         ok = wt.wait(BAR(item_full[slot]), (items >> 1) & 1);
@@ -317,8 +383,8 @@ __global__ void __launch_bounds__(192, 1)
         if (p.debug_stall && !stalled) {
           // test hook: withhold all work of this item until the softmax warps give up
           stalled = true;
-          const uint64_t t0 = ptx::globaltimer();
-          while (!ctl->abort && ptx::globaltimer() - t0 < 4ull * p.wait_limit_ns) {
+          const uint64_t s0 = ptx::globaltimer();
+          while (!ctl->abort && ptx::globaltimer() - s0 < 4ull * p.wait_limit_ns) {
           }
           if (!ctl->abort) wt.give_up();
           ok = false;
@@ -327,34 +393,51 @@ __global__ void __launch_bounds__(192, 1)
         ok = wt.wait(BAR(q_full), qn & 1);
         if (!ok) break;
         ptx::tc_fence_after();
-        for (int idx = 0; idx < it.n && ok; ++idx) {
-          const uint32_t gi = g + idx, kvi = kv + idx;
-          const uint32_t buf = gi & 1, s = kvi & 1;
-          ok = wt.wait(BAR(k_full[s]), (kvi >> 1) & 1);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          const uint32_t k_base = sK + s * C::KV_BYTES;
+        // tiles idx = 0 .. n: QK_idx (idx < n), then PV_{idx-1} (idx >= 1)
+        for (int idx = 0; idx <= it.n && ok; ++idx) {
+          if (idx < it.n) {
+            const uint32_t t = t0 + idx;
+            LITE_TRACE(1, 0, t);
+            if (!wt.wait(BAR(k_full[t & 1]), (t >> 1) & 1)) { ok = false; break; }
+            LITE_TRACE(1, 1, t);
+            ptx::tc_fence_after();
+            const uint64_t kd = k_desc0 + uint64_t(((t & 1) * C::KV_BYTES) >> 4);
+            const uint32_t s_tmem = tmem + C::S_COL + (t & 1) * BN;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk & 3) * 32;  // 16 bf16 = 32 bytes inside the 128-byte swizzle atom
-            const uint64_t adesc = umma_desc_sw128(sQ + (kk >> 2) * C::Q_CHUNK + off, 16, 1024);
-            const uint64_t bdesc = umma_desc_sw128(k_base + (kk >> 2) * C::KV_CHUNK + off, 16, 1024);
-            ptx::mma_ss(tmem + C::S_COL + buf * BN, adesc, bdesc, C::IDESC_QK, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t off = uint64_t((kk >> 2) * (C::Q_CHUNK >> 4) + (kk & 3) * 2);
+              const uint64_t offk = uint64_t((kk >> 2) * (C::KV_CHUNK >> 4) + (kk & 3) * 2);
+              ptx::mma_ss(s_tmem, q_desc + off, kd + offk, C::IDESC_QK, kk > 0 ? 1u : 0u);
+            }
+            ptx::mma_commit(BAR(s_full[t & 1]));
+            LITE_TRACE(1, 2, t);
+            if (idx == it.n - 1) ptx::mma_commit(BAR(q_empty));
           }
-          ptx::mma_commit(BAR(s_full[buf]));
-          ptx::mma_commit(BAR(k_empty[s]));
-          if (idx == it.n - 1) ptx::mma_commit(BAR(q_empty));
           if (idx >= 1) {
-            if (idx == 1 && qn >= 1) ok = wt.wait(BAR(o_free), (qn - 1) & 1);
-            if (ok) ok = issue_pv(gi - 1, kvi - 1, idx == 1);
+            // O_{t%2} += P_t V_t for the previous tile; QK_{t+2} (next iteration but one) reuses
+            // S buffer t%2, and MMAs of this thread run in issue order
+            const int pv = idx - 1;
+            const uint32_t t = t0 + pv;
+            if (pv == 0 && qn >= 1 && !wt.wait(BAR(o_free), (qn - 1) & 1)) { ok = false; break; }
+            LITE_TRACE(1, 3, t);
+            if (!wt.wait(BAR(p_full[t & 1]), (t >> 1) & 1)) { ok = false; break; }
+            LITE_TRACE(1, 4, t);
+            if (!wt.wait(BAR(v_full[t % 3]), (t / 3) & 1)) { ok = false; break; }
+            LITE_TRACE(1, 5, t);
+            ptx::tc_fence_after();
+            const uint32_t p_tmem = tmem + C::S_COL + (t & 1) * BN;
+            const uint32_t o_tmem = tmem + C::O_COL + (t & 1) * D;
+            const uint64_t vd = v_desc0 + uint64_t(((t % 3) * C::KV_BYTES) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk)
+              ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + uint64_t(kk * 128), C::IDESC_PV,
+                          (pv < 2 && kk == 0) ? 0u : 1u);
+            // the epilogue of group t%2 waits for the last PV into its accumulator
+            if (pv >= it.n - 2) ptx::mma_commit(BAR(pv_done[t & 1]));
+            LITE_TRACE(1, 6, t);
           }
         }
-        if (ok) {
-          if (it.n == 1 && qn >= 1) ok = wt.wait(BAR(o_free), (qn - 1) & 1);
-          if (ok) ok = issue_pv(g + it.n - 1, kv + it.n - 1, it.n == 1);
-        }
-        g += it.n;
-        kv += it.n;
+        t0 += it.n;
         ++qn;
       }
       // all issued tensor-core work must finish before TMEM is released
@@ -363,11 +446,13 @@ __global__ void __launch_bounds__(192, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------------------- softmax warps
+    // ------------------------------------------------------------------------- softmax warpgroups
+    const int grp = (warp - 2) >> 2;                // tiles t with t % 2 == grp
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;  // TMEM lane = row inside the tile slot
+    const int r = quarter * 32 + lane;              // TMEM lane = row inside the tile slot
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
-    uint32_t g = 0, items = 0, qn = 0;
+    const uint32_t vote_bar = 1 + grp;              // named barrier of this warpgroup (128 threads)
+    uint32_t t0 = 0, items = 0, pv_phase = 0;
     while (true) {
       const int slot = items & 1;
       bool ok = wt.wait(BAR(item_full[slot]), (items >> 1) & 1);
@@ -375,34 +460,40 @@ __global__ void __launch_bounds__(192, 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(BAR(item_empty[slot]));
       ++items;
-      if (!ptx::named_bar_and(1, 128, ok) || item < 0) break;
+      if (!ptx::named_bar_and(3, 256, ok) || item < 0) break;
       const ItemInfo it = decode_item(p, item);
       const int n_row = it.qi * C::BQ + r;
       const bool valid_row = (r < C::BQ) && (n_row < p.N);
       const size_t o_off = (size_t(it.b) * p.N + n_row) * p.H + it.h;
       if (it.n == 0) {
         if (valid_row) {
-          uint4* dst = reinterpret_cast<uint4*>(p.o + o_off * D);
-          for (int x = 0; x < D / 8; ++x) dst[x] = make_uint4(0, 0, 0, 0);
-          if (p.lse) p.lse[(size_t(it.b) * p.H + it.h) * p.N + n_row] = -INFINITY;
+          uint4* dst = reinterpret_cast<uint4*>(p.o + o_off * D + grp * (D / 2));
+          for (int x = 0; x < D / 16; ++x) dst[x] = make_uint4(0, 0, 0, 0);
+          if (p.lse && grp == 0) p.lse[(size_t(it.b) * p.H + it.h) * p.N + n_row] = -INFINITY;
         }
         continue;
       }
-      float m_true = -INFINITY;  // running max of visited tiles (log2 units)
-      float m_used = -INFINITY;  // max the exponentials are taken against (lazy rescale)
-      float l = 0.f;
-      for (int idx = 0; idx < it.n; ++idx) {
-        const uint32_t gi = g + idx;
-        const uint32_t buf = gi & 1;
-        const int j = key_tile(p, it.row, idx);
-        wt.wait(BAR(s_full[buf]), (gi >> 1) & 1);
+      float m_true = -INFINITY;  // running max over all earlier tiles of the item (log2 units)
+      float m_used = -INFINITY;  // this group's exponent reference (lazy rescale)
+      float l = 0.f;             // this group's share of the row sum
+      // this group's tiles of the item: idx = first, first + 2, ...
+      const int first = int((uint32_t(grp) - t0) & 1u);
+      int j_next = first < it.n ? key_tile(p, it.row, first) : 0;
+      for (int idx = first; idx < it.n; idx += 2) {
+        const uint32_t t = t0 + idx;
+        const int j = j_next;
+        if (idx + 2 < it.n) j_next = key_tile(p, it.row, idx + 2);  // prefetch
+        if (r == 0) LITE_TRACE(2 + grp, 0, t);
+        wt.wait(BAR(s_full[grp]), (t >> 1) & 1);
         __syncwarp();
         ptx::tc_fence_after();
-        const uint32_t s_tmem = tmem + lane_base + C::S_COL + buf * BN;
+        const uint32_t s_tmem = tmem + lane_base + C::S_COL + grp * BN;
         uint32_t sr[BN];
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) ptx::tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        for (int c = 0; c < BN / 32; ++c)
+          ptx::tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
         ptx::tmem_wait_ld();
+        if (r == 0) LITE_TRACE(2 + grp, 1, t);
         float s[BN];
 #pragma unroll
         for (int x = 0; x < BN; ++x) s[x] = __uint_as_float(sr[x]);
@@ -413,19 +504,36 @@ __global__ void __launch_bounds__(192, 1)
           for (int x = 0; x < BN; ++x)
             if (x >= valid_cols) s[x] = -INFINITY;
         }
-        float mx = s[0];
+        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-        for (int x = 1; x < BN; ++x) mx = fmaxf(mx, s[x]);
-        const float loc = mx * p.scale_log2;
+        for (int x = 0; x < BN; x += 8) {
+          m0 = ptx::fmax3(m0, s[x], s[x + 1]);
+          m1 = ptx::fmax3(m1, s[x + 2], s[x + 3]);
+          m2 = ptx::fmax3(m2, s[x + 4], s[x + 5]);
+          m3 = ptx::fmax3(m3, s[x + 6], s[x + 7]);
+        }
+        const float loc = ptx::fmax3(m0, m1, fmaxf(m2, m3)) * p.scale_log2;
+        // post this tile's row maxima for the other group, then fold in the previous tile's
+        if (r == 0) LITE_TRACE(2 + grp, 2, t);
+        mailbox[(t & 3) * 128 + r] = loc;
+        ptx::mbar_arrive(BAR(mx_full[t & 3]));
+        if (idx > 0) {
+          wt.wait(BAR(mx_full[(t - 1) & 3]), ((t - 1) >> 2) & 1);
+          m_true = fmaxf(m_true, mailbox[((t - 1) & 3) * 128 + r]);
+        }
+        if (r == 0) LITE_TRACE(2 + grp, 3, t);
         if (p.skip_test) {
           // QK-Skip: flag tile j when loc - m < tau for every valid row (m over earlier tiles)
           const bool pred = !valid_row || (loc - m_true < p.tau_log2);
-          const bool flag = ptx::named_bar_and(1, 128, pred);
+          const bool flag = ptx::named_bar_and(vote_bar, 128, pred);
           if (flag && r == 0 && p.mask_out && !ctl->abort)
             atomicOr(p.mask_out + size_t(it.row) * p.W + (j >> 5), 1u << (j & 31));
         }
+        if (r == 0) LITE_TRACE(2 + grp, 4, t);
         m_true = fmaxf(m_true, loc);
-        // lazy rescale: move the reference max only when it grew by more than 8 (log2 units)
+        // lazy rescale of this group's accumulator: move the reference only when the tile max
+        // exceeds it by more than 8 (log2 units). The previous PV into this accumulator (tile t-2)
+        // was issued before QK_t, so it has completed now that S_t is ready.
         const bool need = loc > m_used + 8.0f;
         float alpha = 1.f;
         if (need) {
@@ -433,77 +541,118 @@ __global__ void __launch_bounds__(192, 1)
           m_used = loc;
           l *= alpha;
         }
-        const bool warp_need = __any_sync(0xffffffffu, need);
-        // P = 2^(s*scale*log2e - m_used), bf16 pairs written over the consumed S columns
-        const float neg_m = -m_used;
-        float rowsum = 0.f;
+        const bool warp_need = __any_sync(0xffffffffu, need) && (idx >= 2);
+        // P = 2^(s*scale*log2e - m_used) as bf16 pairs, written over S columns already read: the
+        // chunk loop re-reads S 32 columns at a time (compact code, few live registers) and chunk
+        // c's P lands in columns [16c, 16c+16), all read by chunks <= c. Packed fp32x2 arithmetic
+        // for the affine step and the row sum; one column pair in four is exponentiated on the FMA
+        // pipe, the rest on MUFU, to balance the two units and the issue slots.
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 nm2 = make_float2(-m_used, -m_used);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        // one chunk of 32 S columns -> 16 bf16 pairs of P at column 16c
+        auto exp_chunk = [&](const uint32_t (&q)[32], int c) {
+          const int vc = valid_cols - c * 32;  // valid columns in this chunk (>= 32 except in the tail)
+          uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < BN / 64; ++c) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            const float p0 = ptx::ex2(fmaf(s[c * 64 + 2 * x], p.scale_log2, neg_m));
-            const float p1 = ptx::ex2(fmaf(s[c * 64 + 2 * x + 1], p.scale_log2, neg_m));
-            rowsum += p0 + p1;
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+          for (int x = 0; x < 16; ++x) {
+            float s0 = __uint_as_float(q[2 * x]), s1 = __uint_as_float(q[2 * x + 1]);
+            if (vc < 32) {
+              s0 = 2 * x < vc ? s0 : -INFINITY;
+              s1 = 2 * x + 1 < vc ? s1 : -INFINITY;
+            }
+            const float2 a = __ffma2_rn(make_float2(s0, s1), sc2, nm2);
+            const float2 pp = ((x & 3) == 3) ? exp2_poly2(a) : make_float2(ptx::ex2(a.x), ptx::ex2(a.y));
+            acc[x & 3] = __fadd2_rn(acc[x & 3], pp);
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(pp.x, pp.y);
             pk[x] = *reinterpret_cast<uint32_t*>(&h2);
           }
-          ptx::tmem_st32(s_tmem + c * 32, pk);
+          ptx::tmem_st16(s_tmem + c * 16, pk);
+        };
+        // double-buffered: the next chunk's TMEM load is in flight while this chunk is computed
+        // (tcgen05.wait::ld waits for all of this thread's loads, so the next load is issued after it)
+        uint32_t qa[32], qb[32];
+        ptx::tmem_ld32(s_tmem, qa);
+        ptx::tmem_wait_ld();
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; c += 2) {
+          ptx::tmem_ld32(s_tmem + (c + 1) * 32, qb);
+          exp_chunk(qa, c);
+          ptx::tmem_wait_ld();
+          if (c + 2 < BN / 32) ptx::tmem_ld32(s_tmem + (c + 2) * 32, qa);
+          exp_chunk(qb, c + 1);
+          ptx::tmem_wait_ld();
         }
-        l += rowsum;
-        if (idx > 0) {
-          // Every thread observes each PV completion once, in order, so the parity wait is exact.
-          // PV_{gi-1} ran while the exponentials above were computed; O is rescaled only after it.
-          wt.wait(BAR(pv_done), (gi - 1) & 1);
-          __syncwarp();
-          if (warp_need) {
-            ptx::tc_fence_after();
-            const uint32_t o_tmem = tmem + lane_base + C::O_COL;
+        const float2 acc2 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+        l += acc2.x + acc2.y;
+        if (warp_need) {
+          const uint32_t o_tmem = tmem + lane_base + C::O_COL + grp * D;
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t rr[32];
+            ptx::tmem_ld32(o_tmem + c * 32, rr);
+            ptx::tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t rr[32];
-              ptx::tmem_ld32(o_tmem + c * 32, rr);
-              ptx::tmem_wait_ld();
-#pragma unroll
-              for (int x = 0; x < 32; ++x) rr[x] = __float_as_uint(__uint_as_float(rr[x]) * alpha);
-              ptx::tmem_st32(o_tmem + c * 32, rr);
-            }
+            for (int x = 0; x < 32; ++x) rr[x] = __float_as_uint(__uint_as_float(rr[x]) * alpha);
+            ptx::tmem_st32(o_tmem + c * 32, rr);
           }
         }
         ptx::tmem_wait_st();
+        if (r == 0) LITE_TRACE(2 + grp, 6, t);
         ptx::tc_fence_before();
-        ptx::mbar_arrive(BAR(p_full[buf]));
+        ptx::mbar_arrive(BAR(p_full[grp]));
       }
-      // epilogue: wait for the last PV, normalise, store O (bf16) and lse
-      wt.wait(BAR(pv_done), (g + it.n - 1) & 1);
-      __syncwarp();
+      // epilogue: each group waits for its last PV, the two partial softmaxes are combined,
+      // group g stores columns [g*D/2, (g+1)*D/2) of O (bf16) and group 0 the lse
+      if (first < it.n) {
+        wt.wait(BAR(pv_done[grp]), pv_phase & 1);  // one phase per item in which this group has a tile
+        ++pv_phase;
+      }
+      epi[(grp * 2 + 0) * 128 + r] = m_used;
+      epi[(grp * 2 + 1) * 128 + r] = l;
+      ptx::tc_fence_before();
+      ptx::named_bar_sync(3, 256);
       ptx::tc_fence_after();
-      const float inv_l = 1.f / l;
-      const uint32_t o_tmem = tmem + lane_base + C::O_COL;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t rr[32];
-        ptx::tmem_ld32(o_tmem + c * 32, rr);
+      const float mu0 = epi[0 * 128 + r], l0 = epi[1 * 128 + r];
+      const float mu1 = epi[2 * 128 + r], l1 = epi[3 * 128 + r];
+      // group g holds a partial iff it had a tile in this item (both do when n >= 2)
+      const bool has0 = ((0u - t0) & 1u) < uint32_t(it.n);
+      const bool has1 = ((1u - t0) & 1u) < uint32_t(it.n);
+      const float mm = has0 && has1 ? fmaxf(mu0, mu1) : (has0 ? mu0 : mu1);
+      const float a0 = has0 ? ptx::ex2(mu0 - mm) : 0.f;
+      const float a1 = has1 ? ptx::ex2(mu1 - mm) : 0.f;
+      const float lt = a0 * l0 + a1 * l1;
+      const float inv_l = 1.f / lt;
+      const float w0 = a0 * inv_l, w1 = a1 * inv_l;
+#pragma unroll 1
+      for (int c = 0; c < D / 64; ++c) {
+        const int col = grp * (D / 2) + c * 32;
+        uint32_t r0[32], r1[32];
+        ptx::tmem_ld32(tmem + lane_base + C::O_COL + 0 * D + col, r0);
+        ptx::tmem_ld32(tmem + lane_base + C::O_COL + 1 * D + col, r1);
         ptx::tmem_wait_ld();
         if (valid_row) {
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(rr[2 * x]) * inv_l,
-                                                      __uint_as_float(rr[2 * x + 1]) * inv_l);
+            // an accumulator without a partial may hold stale data: select, never multiply by zero
+            const float o0 = (has0 ? w0 * __uint_as_float(r0[2 * x]) : 0.f) +
+                             (has1 ? w1 * __uint_as_float(r1[2 * x]) : 0.f);
+            const float o1 = (has0 ? w0 * __uint_as_float(r0[2 * x + 1]) : 0.f) +
+                             (has1 ? w1 * __uint_as_float(r1[2 * x + 1]) : 0.f);
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(o0, o1);
             pk[x] = *reinterpret_cast<uint32_t*>(&h2);
           }
-          uint4* dst = reinterpret_cast<uint4*>(p.o + o_off * D + c * 32);
+          uint4* dst = reinterpret_cast<uint4*>(p.o + o_off * D + col);
 #pragma unroll
           for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
         }
       }
-      if (valid_row && p.lse)
-        p.lse[(size_t(it.b) * p.H + it.h) * p.N + n_row] = (m_used + __log2f(l)) * 0.6931471805599453f;
+      if (valid_row && grp == 0 && p.lse)
+        p.lse[(size_t(it.b) * p.H + it.h) * p.N + n_row] = (mm + __log2f(lt)) * 0.6931471805599453f;
       ptx::tc_fence_before();
       ptx::mbar_arrive(BAR(o_free));
-      g += it.n;
-      ++qn;
+      t0 += it.n;
     }
   }
 #undef BAR

@@ -31,6 +31,9 @@ struct Options {
 Options g_opt;
 cudaEvent_t g_ev_before = nullptr;
 cudaEvent_t g_ev_after = nullptr;
+#ifdef LITE_ATTN_TRACE
+long long* g_trace = nullptr;
+#endif
 
 struct DeviceCache {
   bool init = false;
@@ -130,7 +133,7 @@ int launch_attention(DeviceCache* dc, int cfg_slot, const void* q, const void* k
   if (p.n_items < grid) grid = p.n_items;
   if (grid <= 0) return LITE_OK;
   if (g_ev_before) cudaEventRecord(g_ev_before, stream);
-  lite::lite_attn_kernel<D, BN><<<grid, 192, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  lite::lite_attn_kernel<D, BN><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
   if (g_ev_after) cudaEventRecord(g_ev_after, stream);
   return LITE_OK;
@@ -159,6 +162,9 @@ lite::AttnParams base_params(void* o, float* lse, int B, int H, int N, int d, fl
   p.status = dc->status;
   p.wait_limit_ns = g_opt.wait_limit_ns;
   p.debug_stall = g_opt.debug_stall;
+#ifdef LITE_ATTN_TRACE
+  p.trace = g_trace;
+#endif
   return p;
 }
 
@@ -323,6 +329,14 @@ int lite_attn_dense(const void* q, const void* k, const void* v, void* o, float*
   // every tile live, identity order, static striding over items (uniform cost): no scratch
   return run_attention(dc, d, q, k, v, p, as_stream(stream));
 }
+
+#ifdef LITE_ATTN_TRACE
+// analysis builds only: clock64 probes of the first CTAs go to this device buffer
+int lite_trace_set(void* buf) {
+  g_trace = static_cast<long long*>(buf);
+  return LITE_OK;
+}
+#endif
 
 }  // extern "C"
 
