@@ -52,6 +52,9 @@ def parse_args():
     ap.add_argument("--tau", type=float, default=None, help="fixed tau instead of the workload's schedule")
     ap.add_argument("--cpu-sample-tiles", type=int, default=24, help="query tiles per step (reference arm)")
     ap.add_argument("--heads", type=int, default=None, help="override H (a smaller layer, e.g. for profiling)")
+    ap.add_argument("--study", choices=["sweep", "stress"], default=None,
+                    help="threshold sweep (720p shape) or stress-workload report instead of the headline line")
+    ap.add_argument("--study-steps", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     return ap.parse_args()
@@ -282,6 +285,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.study:
+        return run_study(args)
 
     from temporal_block_sparse_b200 import lite_attn as la
 
@@ -490,6 +495,131 @@ def run_e2e(args, la, wl, qkv, masks, dev, world, dist):
     value = wl.dense_flop() * len(timed) * world / (ms * 1e-3) / 1e12
     return {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": ms / len(timed), "note": "pinned host q/k/v in, o/lse out; copies overlap compute"}
+
+
+# --------------------------------------------------------------------------------- studies
+
+
+def _time_call(fn, reps=1):
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def _skipped_bound(q, k, mask_in, mask_out, tau, tiles):
+    """For flagged tiles of sampled query tiles: max p / exp(tau) and max row mass / (cols * exp(tau))
+    under that step's dense softmax (oracle arithmetic, float64). Both are < 1 by the QK-Skip rule."""
+    import numpy as np
+
+    B, N, H, d = q.shape
+    tile = 128 if d == 128 else 64
+    scale = 1.0 / math.sqrt(d)
+    before = mask_in.cpu().numpy().view(np.uint32)
+    after = mask_out.cpu().numpy().view(np.uint32)
+    worst_p, worst_mass, n = 0.0, 0.0, 0
+    for (b, h, i) in tiles:
+        r0, r1 = i * tile, min(N, (i + 1) * tile)
+        qi = q[b, r0:r1, h].double().cpu()
+        kk = k[b, :, h].double().cpu()
+        s_ = scale * (qi @ kk.T)
+        p_ = torch.softmax(s_, dim=-1).numpy()
+        new = after[b, h, i] & ~before[b, h, i]
+        for w in range(new.shape[0]):
+            bits = int(new[w])
+            while bits:
+                bit = (bits & -bits).bit_length() - 1
+                bits &= bits - 1
+                j = w * 32 + bit
+                blk = p_[:, j * tile:min(N, (j + 1) * tile)]
+                worst_p = max(worst_p, float(blk.max()) / math.exp(tau))
+                worst_mass = max(worst_mass, float(blk.sum(1).max()) / (blk.shape[1] * math.exp(tau)))
+                n += 1
+    return {"flagged_tiles_checked": n, "max_p_over_exp_tau": worst_p, "max_rowmass_over_cols_exp_tau": worst_mass}
+
+
+def run_study(args):
+    """Threshold sweep and stress reports (one JSON line per run; not the headline metric)."""
+    from temporal_block_sparse_b200 import lite_attn as la
+
+    torch.cuda.set_device(0)
+    la.load()
+    if args.study == "sweep":
+        base = wlmod.WORKLOADS["sweep"]
+        steps = args.study_steps or base.steps
+        taus = wlmod.SWEEP_TAUS
+    else:
+        base = wlmod.WORKLOADS["stress"]
+        steps = args.study_steps or base.steps
+        taus = (-3.0,)
+    B, N, H, d = base.B, base.N, base.H, base.d
+    tile, T, W = la.lite_mask_geometry(N, d)
+    dense_flop = base.dense_flop()
+    # dense reference time on this shape
+    tr = wlmod.Trajectory(base, device="cuda")
+    q, k, v = tr.current()
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    la.lite_attn_dense(q, k, v, o=o, lse=lse)
+    dense_ms = _time_call(lambda: la.lite_attn_dense(q, k, v, o=o, lse=lse), reps=3)
+    del tr, q, k, v
+    for tau in taus:
+        tr = wlmod.Trajectory(base, device="cuda")
+        m_in = torch.zeros((B, H, T, W), dtype=torch.int32, device="cuda")
+        m_out = torch.empty_like(m_in)
+        per_step = []
+        bound = None
+        for t in range(steps):
+            q, k, v = tr.current()
+            frac = skipped_fraction(m_in, T)
+            ex = live_flop(m_in, N, d, tile)
+            # min of two runs of the same step (idempotent: same mask_in, same mask_out)
+            step = lambda: la.lite_attn_fwd(q, k, v, m_in, m_out, tau=tau, o=o, lse=lse)
+            ms = min(_time_call(step), _time_call(step))
+            if t == 0 and math.isfinite(tau) and args.study == "sweep":
+                tiles = [(0, 7, T - 1), (0, 21, T // 2), (0, 33, (3 * T) // 4)]
+                bound = _skipped_bound(q, k, m_in, m_out, tau, tiles)
+            rec = {"step": t, "skipped": frac, "ms": ms, "speedup_vs_dense": dense_ms / ms,
+                   "executed_tflops": ex / (ms * 1e-3) / 1e12, "dense_equiv_tflops": dense_flop / (ms * 1e-3) / 1e12}
+            if args.study == "stress":
+                words = m_in.to(torch.int64) & 0xFFFFFFFF
+                bits = ((words.unsqueeze(-1) >> torch.arange(32, device="cuda")) & 1).reshape(B, H, T, -1)[..., :T]
+                per_head = bits.float().mean(dim=(2, 3)).flatten().cpu()
+                rec["per_head_skipped"] = {"min": float(per_head.min()), "mean": float(per_head.mean()),
+                                           "max": float(per_head.max())}
+                lst = torch.empty((B, H, T, T), dtype=torch.int16, device="cuda")
+                cnt = torch.empty((B, H, T), dtype=torch.int32, device="cuda")
+                ordr = torch.empty(B * H * T, dtype=torch.int32, device="cuda")
+                lib = la.load()
+                sh = torch.cuda.current_stream().cuda_stream
+                rec["compaction_ms"] = _time_call(lambda: lib.lite_mask_to_list(m_in.data_ptr(), lst.data_ptr(),
+                                                                                cnt.data_ptr(), B, H, N, d, sh))
+                rec["schedule_ms"] = _time_call(lambda: lib.lite_schedule(cnt.data_ptr(), ordr.data_ptr(), B, H, T, sh))
+            per_step.append(rec)
+            m_in, m_out = m_out, m_in
+            tr.advance()
+        assert la.lite_get_device_status() == 0
+        # linearity: step time against live fraction (least squares), over steps with any skipping
+        xs = [1 - r["skipped"] for r in per_step]
+        ys = [r["ms"] for r in per_step]
+        fit = None
+        if max(xs) - min(xs) > 0.02:
+            mx, my = sum(xs) / len(xs), sum(ys) / len(ys)
+            sxx = sum((x - mx) ** 2 for x in xs)
+            sxy = sum((x - mx) * (y - my) for x, y in zip(xs, ys))
+            slope = sxy / sxx
+            icpt = my - slope * mx
+            ss_res = sum((y - (icpt + slope * x)) ** 2 for x, y in zip(xs, ys))
+            ss_tot = sum((y - my) ** 2 for y in ys)
+            fit = {"ms_at_live_1": icpt + slope, "ms_at_live_0": icpt, "r2": 1 - ss_res / ss_tot if ss_tot else 1.0}
+        line = {"study": args.study, "workload": f"{base.name}: B={B} H={H} N={N} d={d}", "tau": tau,
+                "steps": steps, "dense_ms": dense_ms, "final_skipped": per_step[-1]["skipped"],
+                "time_vs_live_fraction_fit": fit, "skipped_mass_bound_step0": bound, "per_step": per_step}
+        print(json.dumps(line), flush=True)
+        del tr
 
 
 if __name__ == "__main__":

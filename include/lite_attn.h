@@ -79,7 +79,9 @@ enum {
  *
  * A query tile whose live list is empty (only possible with a caller-built mask) yields o = 0 and
  * lse = -inf for its rows. Scratch memory (per-row live lists and the work order) is taken with
- * cudaMallocAsync on `stream` and released with cudaFreeAsync on the same stream.
+ * cudaMallocFromPoolAsync on `stream` from a stream-ordered pool the library creates per device
+ * (it retains freed memory for reuse; its peak is the largest scratch of any call) and released
+ * with cudaFreeAsync on the same stream.
  * Returns LITE_OK once enqueued; device-side failures are reported by lite_get_device_status().
  */
 int lite_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,

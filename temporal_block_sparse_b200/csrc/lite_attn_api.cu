@@ -40,6 +40,10 @@ struct DeviceCache {
   int sms = 0;
   int* status = nullptr;
   bool smem_set[4] = {false, false, false, false};
+  // Library-owned stream-ordered pool for per-call scratch. It keeps freed memory (release
+  // threshold = max), so steady-state calls reuse it instead of mapping new memory, and it does
+  // not alter the application's default pool.
+  cudaMemPool_t pool = nullptr;
 };
 DeviceCache g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -57,6 +61,14 @@ int device_cache(DeviceCache** out) {
     if (cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return LITE_ERR_CUDA;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&c.status), g_device_status) != cudaSuccess)
       return LITE_ERR_CUDA;
+    cudaMemPoolProps props;
+    std::memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    if (cudaMemPoolCreate(&c.pool, &props) != cudaSuccess) return LITE_ERR_CUDA;
+    uint64_t keep = ~uint64_t(0);
+    if (cudaMemPoolSetAttribute(c.pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) return LITE_ERR_CUDA;
     c.init = true;
   }
   if (!g_encode) {
@@ -284,7 +296,7 @@ int lite_attn_fwd(const void* q, const void* k, const void* v, void* o, float* l
   const size_t ord_b = align256(size_t(rows) * sizeof(int32_t));
   const size_t total = list_b + 2 * cnt_b + 256;
   void* ws = nullptr;
-  if (cudaMallocAsync(&ws, total, s) != cudaSuccess) return LITE_ERR_CUDA;
+  if (cudaMallocFromPoolAsync(&ws, total, dc->pool, s) != cudaSuccess) return LITE_ERR_CUDA;
   char* base = static_cast<char*>(ws);
   int16_t* list = reinterpret_cast<int16_t*>(base);
   int32_t* counts = reinterpret_cast<int32_t*>(base + list_b);
