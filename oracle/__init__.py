@@ -9,6 +9,8 @@ from .lite_attention import (  # noqa: F401
     is_skipped,
     lite_attention_forward,
     live_flop,
+    lse_merge,
+    range_tiles,
     live_key_tiles,
     mask_to_list,
     schedule_order,

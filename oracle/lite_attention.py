@@ -33,9 +33,21 @@ precision of the GPU kernel's scores: each score is rounded to float32 and the m
 compare run in float32. Margins (max_r delta_r - tau) are reported so that tiles within rounding
 distance of tau can be told apart from real disagreements.
 
-Layouts (those of the C ABI): q, k, v [B, N, H, d]; lse [B, H, N] natural log; masks uint32
-[B, H, T, W] with bit (j & 31) of word (j >> 5) set meaning "skip key tile j"; T = ceil(N / tile),
-W = ceil(T / 32). Tile = 64 for d = 64 and 128 for d = 128.
+Layouts (those of the C ABI): q [B, Nq, H, d], k and v [B, Nk, H, d] (Nq = Nk = N for self
+attention); lse [B, H, Nq] natural log; masks uint32 [B, H, Tq, Wk] with bit (j & 31) of word
+(j >> 5) set meaning "skip key tile j"; Tq = ceil(Nq / tile), Tk = ceil(Nk / tile),
+Wk = ceil(Tk / 32). Tile = 64 for d = 64 and 128 for d = 128.
+
+Partial attentions (README, "Both LiteAttention and SeqParallelLiteAttention support returning the
+softmax log-sum-exp (LSE) values for combining results from multiple partial attention
+computations"): outputs over disjoint key sets combine by their LSE -- lse = log sum_p exp(lse_p),
+o = sum_p exp(lse_p - lse) o_p -- which is the softmax over the union of the key sets.
+
+Key-token ranges (README, must_do_list / must_skip_list): a list [start_0, end_0, start_1, end_1,
+...] with start_i > end_i > start_{i+1} names the key tokens end_i + 1 .. start_i (start inclusive,
+end exclusive, counted downwards because the kernel iterates in reverse). A key tile holding any
+must-do token is always live and never flagged; a key tile lying entirely inside must-skip ranges
+is always skipped; must-do wins where both apply.
 """
 
 from __future__ import annotations
@@ -83,6 +95,12 @@ def live_key_tiles(mask: Optional[np.ndarray], b: int, h: int, i: int, T: int) -
     if mask is None:
         return list(range(T - 1, -1, -1))
     return [j for j in range(T - 1, -1, -1) if not is_skipped(mask, b, h, i, j)]
+
+
+def visit_order(tiles) -> List[int]:
+    """Order in which a query tile's live key tiles are visited: highest index first (README,
+    must_do_list: "we iterate in reverse order inside of the kernel")."""
+    return sorted(tiles, reverse=True)
 
 
 def mask_to_list(mask, T: int) -> Tuple[np.ndarray, np.ndarray]:
@@ -137,17 +155,40 @@ class QTileResult:
     margins: Dict[int, float] = field(default_factory=dict)  # j -> max_r delta_r - tau (float64 of fp32)
 
 
+def range_tiles(ranges: Optional[Sequence[int]], Nk: int, tile: int, whole: bool) -> set:
+    """Key tiles touched by a README-style range list (any token if whole=False, all tokens if True)."""
+    out = set()
+    if not ranges:
+        return out
+    r = list(ranges)
+    assert len(r) % 2 == 0, "ranges come in (start, end) pairs"
+    tokens = set()
+    for a, e in zip(r[0::2], r[1::2]):
+        assert a > e, "start_i > end_i (descending convention)"
+        tokens.update(x for x in range(e + 1, a + 1) if 0 <= x < Nk)
+    Tk = (Nk + tile - 1) // tile
+    for j in range(Tk):
+        cols = set(range(j * tile, min(Nk, (j + 1) * tile)))
+        if (cols <= tokens) if whole else (cols & tokens):
+            out.add(j)
+    return out
+
+
 def attend_query_tile(q, k, v, mask_in, b: int, h: int, i: int, tile: int, scale: float,
-                      tau: float, skip_test: bool = True) -> QTileResult:
+                      tau: float, skip_test: bool = True, force_live=frozenset(),
+                      force_skip=frozenset()) -> QTileResult:
     """One query tile of one head: output, LSE and QK-Skip flags.
 
-    q, k, v: float64 arrays [B, N, H, d]. mask_in: uint32 [B,H,T,W] or None (nothing skipped).
+    q: float64 [B, Nq, H, d]; k, v: float64 [B, Nk, H, d]. mask_in: uint32 [B,H,Tq,Wk] or None.
+    force_live / force_skip: key tiles the must-do / must-skip ranges pin.
     """
     N = q.shape[1]
-    T = (N + tile - 1) // tile
+    Nk = k.shape[1]
+    T = (Nk + tile - 1) // tile
     rows = range(i * tile, min(N, (i + 1) * tile))
     d = q.shape[3]
-    live = live_key_tiles(mask_in, b, h, i, T)
+    candidates = {j for j in live_key_tiles(mask_in, b, h, i, T) if j not in force_skip} | set(force_live)
+    live = visit_order(candidates)
     if not live:
         # every key tile skipped: nothing to normalise over
         return QTileResult(b, h, i, rows, np.zeros((len(rows), d)), np.full(len(rows), NEG_INF), [], [], {})
@@ -156,11 +197,11 @@ def attend_query_tile(q, k, v, mask_in, b: int, h: int, i: int, tile: int, scale
     # step 2: scores of the live tiles, scale * q . k, float64
     scores = {}
     for j in live:
-        c0, c1 = j * tile, min(N, (j + 1) * tile)
+        c0, c1 = j * tile, min(Nk, (j + 1) * tile)
         scores[j] = scale * (qi @ k[b, c0:c1, h, :].T)
 
     # step 3: output by its plain definition -- softmax over the union of live columns
-    cols = np.concatenate([np.arange(j * tile, min(N, (j + 1) * tile)) for j in live])
+    cols = np.concatenate([np.arange(j * tile, min(Nk, (j + 1) * tile)) for j in live])
     s_all = np.concatenate([scores[j] for j in live], axis=1)
     row_max = s_all.max(axis=1)
     lse = row_max + np.log(np.exp(s_all - row_max[:, None]).sum(axis=1))
@@ -177,7 +218,7 @@ def attend_query_tile(q, k, v, mask_in, b: int, h: int, i: int, tile: int, scale
             loc = scores[j].astype(np.float32).max(axis=1)
             with np.errstate(invalid="ignore"):
                 delta = loc - m  # +inf where m = -inf
-            if bool(np.all(delta < tau32)):
+            if bool(np.all(delta < tau32)) and j not in force_live:
                 flagged.append(j)
             margins[j] = float(delta.max()) - float(tau)
             m = np.maximum(m, loc)
@@ -195,11 +236,13 @@ class ForwardResult:
 def lite_attention_forward(q, k, v, mask_in=None, scale: Optional[float] = None, tau: float = -10.0,
                            tile: Optional[int] = None,
                            query_tiles: Optional[Iterable[Tuple[int, int, int]]] = None,
-                           skip_test: bool = True) -> ForwardResult:
+                           skip_test: bool = True, must_do=None, must_skip=None) -> ForwardResult:
     """LiteAttention forward for one layer at one denoising step.
 
-    q, k, v: arrays [B, N, H, d] of bf16-representable values (any float dtype; widened to float64).
-    mask_in: uint32/int32 [B, H, T, W] Skip-Mask read at this step, or None for all-live.
+    q: [B, Nq, H, d]; k, v: [B, Nk, H, d] (Nq = Nk for self attention), bf16-representable values
+    (any float dtype; widened to float64).
+    mask_in: uint32/int32 [B, H, Tq, Wk] Skip-Mask read at this step, or None for all-live.
+    must_do / must_skip: README-style key-token range lists, or None.
     scale: softmax scale; None, NaN or <= 0 gives 1/sqrt(d) (the README's Wan2.1 call passes none).
     tau: QK-Skip threshold (natural-log units of scale*QK^T); -inf disables flagging.
     query_tiles: optional list of (b, h, i) to compute (sampled mode); default all.
@@ -210,12 +253,16 @@ def lite_attention_forward(q, k, v, mask_in=None, scale: Optional[float] = None,
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     B, N, H, d = q.shape
-    t, T, W = geometry(N, d, tile)
+    Nk = k.shape[1]
+    t, Tq, _ = geometry(N, d, tile)
+    _, T, W = geometry(Nk, d, tile)
+    force_live = range_tiles(must_do, Nk, t, whole=False)
+    force_skip = range_tiles(must_skip, Nk, t, whole=True)
     if scale is None or not (scale > 0):
         scale = 1.0 / math.sqrt(d)
     if mask_in is None:
         m_in = None
-        mask_out = np.zeros((B, H, T, W), dtype=np.uint32)
+        mask_out = np.zeros((B, H, Tq, W), dtype=np.uint32)
     else:
         m_in = _as_u32(mask_in).copy()
         # bits at or above T in the last word carry no tile; they read as live and are written 0
@@ -223,12 +270,13 @@ def lite_attention_forward(q, k, v, mask_in=None, scale: Optional[float] = None,
             m_in[..., W - 1] &= np.uint32((1 << (T % 32)) - 1)
         mask_out = m_in.copy()
     if query_tiles is None:
-        query_tiles = [(b, h, i) for b in range(B) for h in range(H) for i in range(T)]
+        query_tiles = [(b, h, i) for b in range(B) for h in range(H) for i in range(Tq)]
     out = np.full((B, N, H, d), np.nan)
     lse = np.full((B, H, N), np.nan)
     tiles = {}
     for (b, h, i) in query_tiles:
-        r = attend_query_tile(q, k, v, m_in, b, h, i, t, scale, tau, skip_test=skip_test)
+        r = attend_query_tile(q, k, v, m_in, b, h, i, t, scale, tau, skip_test=skip_test,
+                              force_live=force_live, force_skip=force_skip)
         out[b, r.rows.start:r.rows.stop, h, :] = r.out
         lse[b, h, r.rows.start:r.rows.stop] = r.lse
         for j in r.flagged:
@@ -245,7 +293,7 @@ def dense_attention(q, k, v, scale: Optional[float] = None) -> Tuple[np.ndarray,
     B, N, H, d = q.shape
     if scale is None or not (scale > 0):
         scale = 1.0 / math.sqrt(d)
-    out = np.empty((B, N, H, d))
+    out = np.empty((B, N, H, v.shape[3]))
     lse = np.empty((B, H, N))
     for b in range(B):
         for h in range(H):
@@ -266,3 +314,22 @@ def live_flop(mask, N: int, d: int, tile: Optional[int] = None) -> float:
     size[T - 1] = N - (T - 1) * t
     live = 1.0 - bits.astype(np.float64)
     return float(4.0 * d * np.einsum("bhij,i,j->", live, size, size))
+
+
+def lse_merge(parts: Sequence[Tuple[np.ndarray, np.ndarray]]) -> Tuple[np.ndarray, np.ndarray]:
+    """Combine partial attentions over disjoint key sets by their LSE.
+
+    parts: [(out [B, N, H, d], lse [B, H, N]), ...]. A part whose lse is -inf for a row (no key
+    there) contributes nothing to that row; if every part is -inf the row is 0 with lse -inf.
+    """
+    lses = np.stack([np.asarray(l, dtype=np.float64) for _, l in parts])  # [P, B, H, N]
+    outs = np.stack([np.asarray(o, dtype=np.float64) for o, _ in parts])  # [P, B, N, H, d]
+    mx = lses.max(axis=0)
+    finite = np.isfinite(mx)
+    safe = np.where(finite, mx, 0.0)
+    w = np.where(np.isneginf(lses), 0.0, np.exp(lses - safe[None]))  # [P, B, H, N]
+    tot = w.sum(axis=0)
+    lse = np.where(finite, safe + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    wn = np.where(tot > 0, w / np.where(tot > 0, tot, 1.0)[None], 0.0)  # [P, B, H, N]
+    out = np.einsum("pbhn,pbnhd->bnhd", wn, outs)
+    return out, lse

@@ -98,8 +98,7 @@ def test_planted_ascending_order_is_caught(monkeypatch):
     """Plant a mistake in the oracle (ascending key-tile order); the hand example must reject it."""
     g = _load_golden()
     q, k, v = _golden_inputs(g)
-    orig = ola.live_key_tiles
-    monkeypatch.setattr(ola, "live_key_tiles", lambda *a: list(reversed(orig(*a))))
+    monkeypatch.setattr(ola, "visit_order", lambda tiles: sorted(tiles))
     case = g["cases"][0]
     res = oracle.lite_attention_forward(q, k, v, np.zeros((1, 1, 3, 1), np.uint32), scale=1.0,
                                         tau=case["tau"], tile=2)
@@ -113,8 +112,8 @@ def test_planted_dropped_scale_is_caught(monkeypatch):
     ref_o, ref_l = _brute_head(q[0, :, 0], k[0, :, 0], v[0, :, 0], 1 / 8.0)
     orig = ola.attend_query_tile
 
-    def bad(q_, k_, v_, m_, b, h, i, tile, scale, tau, skip_test=True):
-        return orig(q_, k_, v_, m_, b, h, i, tile, 1.0, tau, skip_test)
+    def bad(q_, k_, v_, m_, b, h, i, tile, scale, tau, skip_test=True, **kw):
+        return orig(q_, k_, v_, m_, b, h, i, tile, 1.0, tau, skip_test, **kw)
 
     monkeypatch.setattr(ola, "attend_query_tile", bad)
     res = oracle.lite_attention_forward(q, k, v, None, tau=-math.inf)
