@@ -19,7 +19,8 @@
  *    between calls (one mask pair per attention layer, README: separate instances per layer).
  *    Device pointers must be device-accessible memory of the current device.
  *  - Layouts:
- *      q, k, v, o : bf16 [B, N, H, d], contiguous, 16-byte aligned. The output o viewed as
+ *      q, k, v, o : bf16 [B, N, H, d], contiguous, 16-byte aligned (cross attention: q and o
+ *                   [B, Nq, H, d], k and v [B, Nk, H, d]). The output o viewed as
  *                   [B, N, H*d] is the README's (batch, seq_len, heads*head_dim) return layout.
  *      lse        : fp32 [B, H, N], natural log of the softmax normaliser of each query row.
  *      masks      : uint32 [B, H, T, W]. Bit (j & 31) of word (j >> 5) set = skip key tile j for
@@ -119,13 +120,15 @@ int lite_mask_to_list(const uint32_t* mask, int16_t* list, int32_t* counts, int 
  * entries (b*H + h)*T + i: a longest-first list schedule that keeps one head's query tiles
  * together so that concurrently running tiles share K/V in L2.
  *
- *  counts  in   device int32 [B, H, T] (from lite_mask_to_list), each in [0, T].
+ *  counts  in   device int32 [B, H, T] (from lite_mask_to_list), each in [0, 4096]. For cross
+ *               attention T here is the number of QUERY tiles (rows per head).
  *  order   out  device int32 [B*H*T].
  *  B*H <= 8192 and T <= 4096 (LITE_ERR_UNSUPPORTED otherwise).
  */
 int lite_schedule(const int32_t* counts, int32_t* order, int B, int H, int T, lite_stream_t stream);
 
-/* Host only: tile edge, tiles per side and mask words per row for (N, d). */
+/* Host only: tile edge, tiles per side and mask words per row for (N, d). For cross attention
+ * call it with Nq for the query-tile count and with Nk for the key-tile count and the words. */
 int lite_mask_geometry(int N, int d, int* tile, int* T, int* words);
 
 /*
@@ -152,7 +155,7 @@ enum { LITE_OPT_WAIT_LIMIT_NS = 1, LITE_OPT_DEBUG_STALL = 2, LITE_OPT_MAX_CTAS =
 int lite_set_option(int option, long long value);
 
 /*
- * lite_set_kernel_events -- measurement hook. While set, every lite_attn_fwd / lite_attn_dense
+ * lite_set_kernel_events -- measurement hook. While set, every lite_attn_fwd* / lite_attn_dense*
  * call records `before` immediately before and `after` immediately after its attention kernel, on
  * the call's stream. Both are cudaEvent_t handles owned by the caller; pass NULL, NULL to stop.
  */
@@ -189,6 +192,74 @@ int lite_set_kernel_events(void* before, void* after);
 int lite_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                           const uint32_t* mask_in, uint32_t* mask_out, int B, int H, int N, int d,
                           float scale, float tau, lite_stream_t stream);
+
+/*
+ * lite_attn_fwd_ex -- lite_attn_fwd for partial attention: queries and keys of different lengths,
+ * plus must-do / must-skip key-token ranges.
+ *
+ * Partial attention (README, LSE section): full self-attention over text and video tokens splits
+ * into text-to-text, text-to-video, video-to-text and video-to-video pieces whose outputs combine
+ * exactly by their LSE (lite_lse_merge). Each piece is this call with its own queries (Nq rows) and
+ * keys / values (Nk rows); the skip test runs only where mask_out is given and tau > -inf (README:
+ * skipping on for video-to-video, off for the others).
+ *
+ * Ranges (README, must_do_list / must_skip_list): a list [start_0, end_0, start_1, end_1, ...] of
+ * key-token indices with start_0 > end_0 > start_1 > end_1 > ... (strictly descending, because
+ * the key tiles are visited in reverse order) names the tokens end_i + 1 .. start_i of each pair
+ * (start inclusive, end exclusive). Tokens at or beyond Nk are ignored.
+ *   - A key tile holding at least one must-do token is live for every query tile whatever the
+ *     mask says, and is never flagged (its mask_out bit is mask_in's).
+ *   - A key tile whose tokens all lie inside must-skip ranges is skipped for every query tile (it
+ *     is not added to mask_out either: the ranges are re-applied on every call).
+ *   - Where both apply, must-do wins.
+ *
+ *  q          in   device bf16 [B, Nq, H, d].
+ *  k, v       in   device bf16 [B, Nk, H, d].
+ *  o          out  device bf16 [B, Nq, H, d].
+ *  lse        out  device fp32 [B, H, Nq], or NULL.
+ *  mask_in    in   device uint32 [B, H, Tq, Wk], or NULL = nothing skipped. Tq = ceil(Nq / tile),
+ *                  Tk = ceil(Nk / tile), Wk = ceil(Tk / 32); bit j of a row = skip key tile j.
+ *  mask_out   out  device uint32 [B, H, Tq, Wk], or NULL; may equal mask_in.
+ *  must_do    in   HOST int32 array of n_must_do entries (even, >= 0), or NULL when n_must_do = 0.
+ *  must_skip  in   HOST int32 array of n_must_skip entries, same convention.
+ *                  The lists are read during the call only. A list that is not strictly
+ *                  descending, has an odd length, or has an end below -1 is LITE_ERR_INVALID_ARG.
+ *  B, H, Nq, Nk, d  Tq, Tk <= 4096; B*H <= 8192; d in {64, 128}.
+ *  scale, tau, stream  as in lite_attn_fwd.
+ * Scratch as in lite_attn_fwd (Tk entries per query tile in the live lists). lite_attn_fwd is this
+ * call with Nq = Nk = N and no ranges.
+ */
+int lite_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                     const uint32_t* mask_in, uint32_t* mask_out, const int32_t* must_do,
+                     int n_must_do, const int32_t* must_skip, int n_must_skip, int B, int H, int Nq,
+                     int Nk, int d, float scale, float tau, lite_stream_t stream);
+
+/*
+ * lite_attn_dense_ex -- lite_attn_dense with Nq query rows and Nk key rows (layouts as in
+ * lite_attn_fwd_ex): the no-skip pieces of a partial attention. No mask, no scratch.
+ */
+int lite_attn_dense_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int H, int Nq, int Nk, int d, float scale, lite_stream_t stream);
+
+/*
+ * lite_lse_merge -- combine partial attentions over disjoint key sets (README, LSE section: the
+ * partial results are combined with their LSE values).
+ *
+ * For every (b, h) and query row n, with parts p = 0 .. n_parts-1:
+ *   lse = ln sum_p exp(lse_p),   o = sum_p exp(lse_p - lse) * o_p,
+ * computed in fp32 from the bf16 partial outputs. Parts with lse_p = -inf for a row contribute
+ * nothing; a row that is -inf in every part gets o = 0 and lse = -inf.
+ *
+ *  outs     in   HOST array of n_parts device pointers, each bf16 [B, N, H, d], 16-byte aligned.
+ *  lses     in   HOST array of n_parts device pointers, each fp32 [B, H, N] (none NULL).
+ *  n_parts       1 .. 8.
+ *  o        out  device bf16 [B, N, H, d]; may be one of outs (in place).
+ *  lse      out  device fp32 [B, H, N], or NULL; may be one of lses.
+ *  B, H, N, d    d in {64, 128}.
+ * The two host arrays are read during the call only.
+ */
+int lite_lse_merge(const void* const* outs, const float* const* lses, int n_parts, void* o,
+                   float* lse, int B, int H, int N, int d, lite_stream_t stream);
 
 #ifdef __cplusplus
 }

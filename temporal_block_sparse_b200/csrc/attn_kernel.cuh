@@ -4,6 +4,9 @@
 // it streams only the live key tiles of that query tile (LiteAttention README, "Full-Stage
 // Elimination": a skipped tile costs no K/V load, no QK^T, no softmax, no PV), from the highest
 // key-tile index down (README, must_do_list: "we iterate in reverse order inside of the kernel").
+// Queries and keys may differ in length (README, LSE section: partial attentions such as text-to-
+// video over a subset of the keys); a key tile that a must-do range keeps live carries a tag in its
+// list entry and is computed but never flagged.
 //
 // Warp roles (320 threads):
 //   warp 0       TMA producer: Q once per item; per live tile K_j into a 2-stage ring and V_j into
@@ -38,17 +41,24 @@ namespace lite {
 
 constexpr int kStatusTimeout = -4;  // LITE_ERR_TIMEOUT
 
+// Skip-List entries are key-tile indices (< 4096). Bit 14 marks a tile that a must-do range keeps
+// live: it is computed like any other tile but never flagged.
+constexpr int kListIndexMask = 0x0fff;
+constexpr int kListNoFlag = 0x4000;
+
 struct AttnParams {
-  __nv_bfloat16* o;         // [B, N, H, D]
-  float* lse;               // [B, H, N] or null
-  uint32_t* mask_out;       // [B, H, T, W] or null (flags not recorded)
-  const int16_t* list;      // [B*H*T, T] live key tiles, descending (null: all tiles, dense)
-  const int32_t* counts;    // [B*H*T] live counts (null: T each)
-  const int32_t* order;     // [B*H*T] work order (null: identity)
+  __nv_bfloat16* o;         // [B, Nq, H, D]
+  float* lse;               // [B, H, Nq] or null
+  uint32_t* mask_out;       // [B, H, Tq, W] or null (flags not recorded)
+  const int16_t* list;      // [B*H*Tq, Tk] live key tiles, descending (null: all tiles, dense)
+  const int32_t* counts;    // [B*H*Tq] live counts (null: Tk each)
+  const int32_t* order;     // [B*H*Tq] work order (null: identity)
   int32_t* work_counter;    // zero before launch; null = static striding over items
   int* status;              // device status word
-  int B, H, N, T, W;
-  int n_items;
+  int B, H;
+  int Nq, Nk;               // query / key tokens (equal for self attention)
+  int Tq, Tk, W;            // query tiles, key tiles, mask words per query tile (ceil(Tk / 32))
+  int n_items;              // B * H * Tq
   float scale_log2;         // softmax scale * log2(e)
   float tau_log2;           // QK-Skip threshold * log2(e)
   int skip_test;            // 1: run the QK-Skip vote and record flags
@@ -207,7 +217,7 @@ struct Waiter {
 };
 
 struct ItemInfo {
-  int row;  // (b*H + h)*T + qi
+  int row;  // (b*H + h)*Tq + qi
   int n;    // live key tiles
   int b, h, qi;
 };
@@ -215,16 +225,17 @@ struct ItemInfo {
 __device__ __forceinline__ ItemInfo decode_item(const AttnParams& p, int item) {
   ItemInfo it;
   it.row = p.order ? p.order[item] : item;
-  it.n = p.counts ? p.counts[it.row] : p.T;
-  const int bh = it.row / p.T;
-  it.qi = it.row - bh * p.T;
+  it.n = p.counts ? p.counts[it.row] : p.Tk;
+  const int bh = it.row / p.Tq;
+  it.qi = it.row - bh * p.Tq;
   it.b = bh / p.H;
   it.h = bh - it.b * p.H;
   return it;
 }
 
-__device__ __forceinline__ int key_tile(const AttnParams& p, int row, int idx) {
-  return p.list ? int(p.list[size_t(row) * p.T + idx]) : (p.T - 1 - idx);
+// idx-th live key tile of a row, with its kListNoFlag tag (dense: Tk-1, Tk-2, ..., untagged)
+__device__ __forceinline__ int key_entry(const AttnParams& p, int row, int idx) {
+  return p.list ? int(p.list[size_t(row) * p.Tk + idx]) : (p.Tk - 1 - idx);
 }
 
 template <int D, int BN>
@@ -320,7 +331,7 @@ __global__ void __launch_bounds__(320, 1)
         q_par = qn & 1;
         ++qn;
         for (int idx = 0; idx < it.n && ok; ++idx, ++t) {
-          const int j = key_tile(p, it.row, idx);
+          const int j = key_entry(p, it.row, idx) & kListIndexMask;
           // K stage t%2 is free once QK_{t-2} finished. V stage t%3 is free once PV_{t-3} finished,
           // which is implied by QK_{t-1} finishing: the MMA thread issues PV_{t-3} before QK_{t-1}
           // and a commit covers every earlier MMA. The s_full barrier of a buffer can only move past
@@ -463,13 +474,13 @@ __global__ void __launch_bounds__(320, 1)
       if (!ptx::named_bar_and(3, 256, ok) || item < 0) break;
       const ItemInfo it = decode_item(p, item);
       const int n_row = it.qi * C::BQ + r;
-      const bool valid_row = (r < C::BQ) && (n_row < p.N);
-      const size_t o_off = (size_t(it.b) * p.N + n_row) * p.H + it.h;
+      const bool valid_row = (r < C::BQ) && (n_row < p.Nq);
+      const size_t o_off = (size_t(it.b) * p.Nq + n_row) * p.H + it.h;
       if (it.n == 0) {
         if (valid_row) {
           uint4* dst = reinterpret_cast<uint4*>(p.o + o_off * D + grp * (D / 2));
           for (int x = 0; x < D / 16; ++x) dst[x] = make_uint4(0, 0, 0, 0);
-          if (p.lse && grp == 0) p.lse[(size_t(it.b) * p.H + it.h) * p.N + n_row] = -INFINITY;
+          if (p.lse && grp == 0) p.lse[(size_t(it.b) * p.H + it.h) * p.Nq + n_row] = -INFINITY;
         }
         continue;
       }
@@ -478,11 +489,12 @@ __global__ void __launch_bounds__(320, 1)
       float l = 0.f;             // this group's share of the row sum
       // this group's tiles of the item: idx = first, first + 2, ...
       const int first = int((uint32_t(grp) - t0) & 1u);
-      int j_next = first < it.n ? key_tile(p, it.row, first) : 0;
+      int j_next = first < it.n ? key_entry(p, it.row, first) : 0;
       for (int idx = first; idx < it.n; idx += 2) {
         const uint32_t t = t0 + idx;
-        const int j = j_next;
-        if (idx + 2 < it.n) j_next = key_tile(p, it.row, idx + 2);  // prefetch
+        const int j = j_next & kListIndexMask;
+        const bool may_flag = !(j_next & kListNoFlag);
+        if (idx + 2 < it.n) j_next = key_entry(p, it.row, idx + 2);  // prefetch
         if (r == 0) LITE_TRACE(2 + grp, 0, t);
         wt.wait(BAR(s_full[grp]), (t >> 1) & 1);
         __syncwarp();
@@ -497,9 +509,9 @@ __global__ void __launch_bounds__(320, 1)
         float s[BN];
 #pragma unroll
         for (int x = 0; x < BN; ++x) s[x] = __uint_as_float(sr[x]);
-        const int valid_cols = min(BN, p.N - j * BN);
+        const int valid_cols = min(BN, p.Nk - j * BN);
         if (valid_cols < BN) {
-          // key columns past N (zero-filled by TMA) take no part in max, sum or PV
+          // key columns past Nk (zero-filled by TMA) take no part in max, sum or PV
 #pragma unroll
           for (int x = 0; x < BN; ++x)
             if (x >= valid_cols) s[x] = -INFINITY;
@@ -526,7 +538,7 @@ __global__ void __launch_bounds__(320, 1)
           // QK-Skip: flag tile j when loc - m < tau for every valid row (m over earlier tiles)
           const bool pred = !valid_row || (loc - m_true < p.tau_log2);
           const bool flag = ptx::named_bar_and(vote_bar, 128, pred);
-          if (flag && r == 0 && p.mask_out && !ctl->abort)
+          if (flag && may_flag && r == 0 && p.mask_out && !ctl->abort)
             atomicOr(p.mask_out + size_t(it.row) * p.W + (j >> 5), 1u << (j & 31));
         }
         if (r == 0) LITE_TRACE(2 + grp, 4, t);
@@ -649,7 +661,7 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       if (valid_row && grp == 0 && p.lse)
-        p.lse[(size_t(it.b) * p.H + it.h) * p.N + n_row] = (mm + __log2f(lt)) * 0.6931471805599453f;
+        p.lse[(size_t(it.b) * p.H + it.h) * p.Nq + n_row] = (mm + __log2f(lt)) * 0.6931471805599453f;
       ptx::tc_fence_before();
       ptx::mbar_arrive(BAR(o_free));
       t0 += it.n;

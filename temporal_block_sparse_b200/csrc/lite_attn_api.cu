@@ -1,12 +1,14 @@
 // lite_attn_api.cu -- host side of the C ABI declared in include/lite_attn.h.
 //
 // Validates arguments (before any CUDA call), builds the TMA tensor maps, takes stream-ordered
-// scratch memory and enqueues: compaction (Skip-Mask -> Skip-List, mask copy) -> schedule (LPT
-// work order) -> persistent attention. Status words, options and per-device caches live here.
+// scratch memory and enqueues: compaction (Skip-Mask -> Skip-List, mask copy, must-do / must-skip
+// ranges) -> schedule (LPT work order) -> persistent attention. Also the LSE merge of partial
+// attentions. Status words, options and per-device caches live here.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -15,6 +17,7 @@
 #include "attn_kernel.cuh"
 #include "lite_attn.h"
 #include "mask_kernels.cuh"
+#include "merge_kernel.cuh"
 
 namespace {
 
@@ -92,15 +95,18 @@ int tile_for(int d) { return d == 64 ? 64 : (d == 128 ? 128 : 0); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int check_shapes(int B, int H, int N, int d) {
-  if (B <= 0 || H <= 0 || N <= 0) return LITE_ERR_INVALID_ARG;
+int check_shapes(int B, int H, int Nq, int Nk, int d) {
+  if (B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0) return LITE_ERR_INVALID_ARG;
   const int t = tile_for(d);
   if (!t) return LITE_ERR_UNSUPPORTED;
-  const long long T = (static_cast<long long>(N) + t - 1) / t;
-  if (T > kMaxT) return LITE_ERR_UNSUPPORTED;
-  if (static_cast<long long>(B) * H * T > (1ll << 30)) return LITE_ERR_UNSUPPORTED;
+  const long long Tq = (static_cast<long long>(Nq) + t - 1) / t;
+  const long long Tk = (static_cast<long long>(Nk) + t - 1) / t;
+  if (Tq > kMaxT || Tk > kMaxT) return LITE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * Tq > (1ll << 30)) return LITE_ERR_UNSUPPORTED;
   return LITE_OK;
 }
+
+int check_shapes(int B, int H, int N, int d) { return check_shapes(B, H, N, N, d); }
 
 int check_qkvo(const void* q, const void* k, const void* v, const void* o, const float* lse) {
   if (!q || !k || !v || !o) return LITE_ERR_INVALID_ARG;
@@ -137,8 +143,8 @@ int launch_attention(DeviceCache* dc, int cfg_slot, const void* q, const void* k
     dc->smem_set[cfg_slot] = true;
   }
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, p.B, p.N, p.H, D, C::BQ) || !make_tmap(&tk, k, p.B, p.N, p.H, D, BN) ||
-      !make_tmap(&tv, v, p.B, p.N, p.H, D, BN))
+  if (!make_tmap(&tq, q, p.B, p.Nq, p.H, D, C::BQ) || !make_tmap(&tk, k, p.B, p.Nk, p.H, D, BN) ||
+      !make_tmap(&tv, v, p.B, p.Nk, p.H, D, BN))
     return LITE_ERR_CUDA;
   int grid = dc->sms;
   if (g_opt.max_ctas > 0 && g_opt.max_ctas < grid) grid = g_opt.max_ctas;
@@ -157,7 +163,8 @@ int run_attention(DeviceCache* dc, int d, const void* q, const void* k, const vo
   return launch_attention<128, 128>(dc, 1, q, k, v, p, stream);
 }
 
-lite::AttnParams base_params(void* o, float* lse, int B, int H, int N, int d, float scale, DeviceCache* dc) {
+lite::AttnParams base_params(void* o, float* lse, int B, int H, int Nq, int Nk, int d, float scale,
+                             DeviceCache* dc) {
   lite::AttnParams p;
   std::memset(&p, 0, sizeof(p));
   const int t = tile_for(d);
@@ -165,10 +172,12 @@ lite::AttnParams base_params(void* o, float* lse, int B, int H, int N, int d, fl
   p.lse = lse;
   p.B = B;
   p.H = H;
-  p.N = N;
-  p.T = (N + t - 1) / t;
-  p.W = (p.T + 31) / 32;
-  p.n_items = B * H * p.T;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.Tq = (Nq + t - 1) / t;
+  p.Tk = (Nk + t - 1) / t;
+  p.W = (p.Tk + 31) / 32;
+  p.n_items = B * H * p.Tq;
   p.scale_log2 = resolve_scale(scale, d) * 1.4426950408889634f;
   p.tau_log2 = -INFINITY;
   p.status = dc->status;
@@ -181,6 +190,120 @@ lite::AttnParams base_params(void* o, float* lse, int B, int H, int N, int d, fl
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ---- the masked forward pass, shared by lite_attn_fwd, lite_attn_fwd_ex and lite_attn_fwd_noalloc
+
+struct FwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  const uint32_t* mask_in;
+  uint32_t* mask_out;
+  int B, H, Nq, Nk, d;
+  float scale, tau;
+};
+
+// every argument check that needs no CUDA call
+int validate_fwd(const FwdArgs& a) {
+  int st = check_qkvo(a.q, a.k, a.v, a.o, a.lse);
+  if (st) return st;
+  st = check_shapes(a.B, a.H, a.Nq, a.Nk, a.d);
+  if (st) return st;
+  if (std::isnan(a.tau)) return LITE_ERR_INVALID_ARG;
+  if (a.tau > 0.f && !debug_env()) return LITE_ERR_INVALID_ARG;
+  if ((a.mask_in && (reinterpret_cast<uintptr_t>(a.mask_in) & 3u)) ||
+      (a.mask_out && (reinterpret_cast<uintptr_t>(a.mask_out) & 3u)))
+    return LITE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(a.B) * a.H > 8192) return LITE_ERR_UNSUPPORTED;
+  return LITE_OK;
+}
+
+// Scratch layout: live lists [rows, Tk] int16 | counts [rows] | order [rows] | work counter.
+struct FwdScratch {
+  size_t list_b, cnt_b, total;
+};
+
+FwdScratch fwd_scratch(const FwdArgs& a) {
+  const int t = tile_for(a.d);
+  const size_t Tq = (a.Nq + t - 1) / t, Tk = (a.Nk + t - 1) / t;
+  const size_t rows = size_t(a.B) * a.H * Tq;
+  FwdScratch f;
+  f.list_b = align256(rows * Tk * sizeof(int16_t));
+  f.cnt_b = align256(rows * sizeof(int32_t));
+  f.total = f.list_b + 2 * f.cnt_b + 256;
+  return f;
+}
+
+// README-style range list -> key-tile bitmap. whole = false: tiles holding any listed token
+// (must-do); whole = true: tiles all of whose tokens are listed (must-skip). The list must be
+// strictly descending (start_0 > end_0 > start_1 > ...), of even length, with ends >= -1; the
+// strict order leaves at least one unlisted token between two ranges, so a tile covered by the
+// union of the ranges is covered by one of them.
+int range_bits(const int32_t* r, int n, int Nk, int t, bool whole, uint32_t* bits) {
+  if (n < 0 || (n & 1) || (n > 0 && !r)) return LITE_ERR_INVALID_ARG;
+  for (int x = 1; x < n; ++x)
+    if (!(r[x - 1] > r[x])) return LITE_ERR_INVALID_ARG;
+  if (n > 0 && r[n - 1] < -1) return LITE_ERR_INVALID_ARG;
+  for (int x = 0; x < n; x += 2) {
+    const long long lo = std::max(static_cast<long long>(r[x + 1]) + 1, 0ll);
+    const long long hi = std::min(static_cast<long long>(r[x]), static_cast<long long>(Nk) - 1);
+    if (lo > hi) continue;
+    for (long long j = lo / t; j <= hi / t; ++j) {
+      if (whole) {
+        const long long c0 = j * t, c1 = std::min((j + 1) * t, static_cast<long long>(Nk)) - 1;
+        if (c0 < lo || c1 > hi) continue;
+      }
+      bits[j >> 5] |= 1u << (j & 31);
+    }
+  }
+  return LITE_OK;
+}
+
+// Enqueues compaction, schedule and attention with the given scratch (fwd_scratch layout).
+int enqueue_fwd(DeviceCache* dc, const FwdArgs& a, const lite::RangeBits* ranges, char* base, cudaStream_t s) {
+  const FwdScratch f = fwd_scratch(a);
+  lite::AttnParams p = base_params(a.o, a.lse, a.B, a.H, a.Nq, a.Nk, a.d, a.scale, dc);
+  const int Tq = p.Tq, Tk = p.Tk, W = p.W, rows = p.n_items;
+  int16_t* list = reinterpret_cast<int16_t*>(base);
+  int32_t* counts = reinterpret_cast<int32_t*>(base + f.list_b);
+  int32_t* order = reinterpret_cast<int32_t*>(base + f.list_b + f.cnt_b);
+  int32_t* counter = reinterpret_cast<int32_t*>(base + f.list_b + 2 * f.cnt_b);
+
+  // the work counter must start at zero (fixed scratch keeps the previous call's value)
+  if (cudaMemsetAsync(counter, 0, sizeof(int32_t), s) != cudaSuccess) return LITE_ERR_CUDA;
+  const int cblocks = (rows + 7) / 8;
+  if (ranges)
+    lite::lite_compact_kernel<true><<<cblocks, 256, 0, s>>>(a.mask_in, a.mask_out, list, counts, rows, Tk, W, *ranges);
+  else
+    lite::lite_compact_kernel<false><<<cblocks, 256, 0, s>>>(a.mask_in, a.mask_out, list, counts, rows, Tk, W,
+                                                             lite::RangeBits{});
+  if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
+  const size_t sm = size_t(a.B * a.H + Tq) * sizeof(int32_t);
+  lite::lite_schedule_kernel<<<a.B * a.H, 512, sm, s>>>(counts, order, a.B * a.H, Tq);
+  if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
+  p.mask_out = a.mask_out;
+  p.list = list;
+  p.counts = counts;
+  p.order = order;
+  p.work_counter = counter;
+  p.tau_log2 = a.tau * 1.4426950408889634f;
+  p.skip_test = (a.mask_out != nullptr && a.tau > -INFINITY) ? 1 : 0;
+  return run_attention(dc, a.d, a.q, a.k, a.v, p, s);
+}
+
+// pool-backed scratch around enqueue_fwd
+int fwd_pooled(const FwdArgs& a, const lite::RangeBits* ranges, cudaStream_t s) {
+  DeviceCache* dc = nullptr;
+  if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
+  const FwdScratch f = fwd_scratch(a);
+  void* ws = nullptr;
+  if (cudaMallocFromPoolAsync(&ws, f.total, dc->pool, s) != cudaSuccess) return LITE_ERR_CUDA;
+  int st = enqueue_fwd(dc, a, ranges, static_cast<char*>(ws), s);
+  if (cudaFreeAsync(ws, s) != cudaSuccess && !st) st = LITE_ERR_CUDA;
+  return st;
+}
 
 }  // namespace
 
@@ -258,7 +381,8 @@ int lite_mask_to_list(const uint32_t* mask, int16_t* list, int32_t* counts, int 
   if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
   const int t = tile_for(d), T = (N + t - 1) / t, W = (T + 31) / 32;
   const int rows = B * H * T;
-  lite::lite_compact_kernel<<<(rows + 7) / 8, 256, 0, as_stream(stream)>>>(mask, nullptr, list, counts, rows, T, W);
+  lite::lite_compact_kernel<false><<<(rows + 7) / 8, 256, 0, as_stream(stream)>>>(mask, nullptr, list, counts, rows,
+                                                                                  T, W, lite::RangeBits{});
   return cudaGetLastError() == cudaSuccess ? LITE_OK : LITE_ERR_CUDA;
 }
 
@@ -275,71 +399,82 @@ int lite_schedule(const int32_t* counts, int32_t* order, int B, int H, int T, li
 
 int lite_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const uint32_t* mask_in,
                   uint32_t* mask_out, int B, int H, int N, int d, float scale, float tau, lite_stream_t stream) {
+  const FwdArgs a{q, k, v, o, lse, mask_in, mask_out, B, H, N, N, d, scale, tau};
+  const int st = validate_fwd(a);
+  if (st) return st;
+  return fwd_pooled(a, nullptr, as_stream(stream));
+}
+
+int lite_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, const uint32_t* mask_in,
+                     uint32_t* mask_out, const int32_t* must_do, int n_must_do, const int32_t* must_skip,
+                     int n_must_skip, int B, int H, int Nq, int Nk, int d, float scale, float tau,
+                     lite_stream_t stream) {
+  const FwdArgs a{q, k, v, o, lse, mask_in, mask_out, B, H, Nq, Nk, d, scale, tau};
+  int st = validate_fwd(a);
+  if (st) return st;
+  lite::RangeBits rb;
+  std::memset(&rb, 0, sizeof(rb));
+  const int t = tile_for(d);
+  st = range_bits(must_do, n_must_do, Nk, t, false, rb.live);
+  if (st) return st;
+  st = range_bits(must_skip, n_must_skip, Nk, t, true, rb.skip);
+  if (st) return st;
+  for (int w = 0; w < 128; ++w) rb.skip[w] &= ~rb.live[w];  // must-do wins
+  const bool any = n_must_do > 0 || n_must_skip > 0;
+  return fwd_pooled(a, any ? &rb : nullptr, as_stream(stream));
+}
+
+int lite_attn_dense_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                       int Nk, int d, float scale, lite_stream_t stream) {
   int st = check_qkvo(q, k, v, o, lse);
   if (st) return st;
-  st = check_shapes(B, H, N, d);
+  st = check_shapes(B, H, Nq, Nk, d);
   if (st) return st;
-  if (std::isnan(tau)) return LITE_ERR_INVALID_ARG;
-  if (tau > 0.f && !debug_env()) return LITE_ERR_INVALID_ARG;
-  if ((mask_in && (reinterpret_cast<uintptr_t>(mask_in) & 3u)) || (mask_out && (reinterpret_cast<uintptr_t>(mask_out) & 3u)))
-    return LITE_ERR_UNSUPPORTED;
-  if (static_cast<long long>(B) * H > 8192) return LITE_ERR_UNSUPPORTED;
   DeviceCache* dc = nullptr;
   if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
-  cudaStream_t s = as_stream(stream);
-  lite::AttnParams p = base_params(o, lse, B, H, N, d, scale, dc);
-  const int T = p.T, W = p.W, rows = p.n_items;
-
-  // scratch: live lists, counts, order, work counter
-  const size_t list_b = align256(size_t(rows) * T * sizeof(int16_t));
-  const size_t cnt_b = align256(size_t(rows) * sizeof(int32_t));
-  const size_t ord_b = align256(size_t(rows) * sizeof(int32_t));
-  const size_t total = list_b + 2 * cnt_b + 256;
-  void* ws = nullptr;
-  if (cudaMallocFromPoolAsync(&ws, total, dc->pool, s) != cudaSuccess) return LITE_ERR_CUDA;
-  char* base = static_cast<char*>(ws);
-  int16_t* list = reinterpret_cast<int16_t*>(base);
-  int32_t* counts = reinterpret_cast<int32_t*>(base + list_b);
-  int32_t* order = reinterpret_cast<int32_t*>(base + list_b + cnt_b);
-  int32_t* counter = reinterpret_cast<int32_t*>(base + list_b + cnt_b + ord_b);
-  (void)ord_b;
-
-  st = LITE_OK;
-  if (cudaMemsetAsync(counter, 0, sizeof(int32_t), s) != cudaSuccess) st = LITE_ERR_CUDA;
-  if (!st) {
-    lite::lite_compact_kernel<<<(rows + 7) / 8, 256, 0, s>>>(mask_in, mask_out, list, counts, rows, T, W);
-    if (cudaGetLastError() != cudaSuccess) st = LITE_ERR_CUDA;
-  }
-  if (!st) {
-    const size_t sm = size_t(B * H + T) * sizeof(int32_t);
-    lite::lite_schedule_kernel<<<B * H, 512, sm, s>>>(counts, order, B * H, T);
-    if (cudaGetLastError() != cudaSuccess) st = LITE_ERR_CUDA;
-  }
-  if (!st) {
-    p.mask_out = mask_out;
-    p.list = list;
-    p.counts = counts;
-    p.order = order;
-    p.work_counter = counter;
-    p.tau_log2 = tau * 1.4426950408889634f;
-    p.skip_test = (mask_out != nullptr && tau > -INFINITY) ? 1 : 0;
-    st = run_attention(dc, d, q, k, v, p, s);
-  }
-  if (cudaFreeAsync(ws, s) != cudaSuccess && !st) st = LITE_ERR_CUDA;
-  return st;
+  lite::AttnParams p = base_params(o, lse, B, H, Nq, Nk, d, scale, dc);
+  // every tile live, identity order, static striding over items (uniform cost): no scratch
+  return run_attention(dc, d, q, k, v, p, as_stream(stream));
 }
 
 int lite_attn_dense(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                     float scale, lite_stream_t stream) {
-  int st = check_qkvo(q, k, v, o, lse);
-  if (st) return st;
-  st = check_shapes(B, H, N, d);
-  if (st) return st;
+  return lite_attn_dense_ex(q, k, v, o, lse, B, H, N, N, d, scale, stream);
+}
+
+int lite_lse_merge(const void* const* outs, const float* const* lses, int n_parts, void* o, float* lse, int B,
+                   int H, int N, int d, lite_stream_t stream) {
+  if (!outs || !lses || !o || n_parts < 1 || B <= 0 || H <= 0 || N <= 0) return LITE_ERR_INVALID_ARG;
+  if (n_parts > lite::kMaxMergeParts) return LITE_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return LITE_ERR_UNSUPPORTED;
+  lite::MergeParts mp;
+  std::memset(&mp, 0, sizeof(mp));
+  for (int x = 0; x < n_parts; ++x) {
+    if (!outs[x] || !lses[x]) return LITE_ERR_INVALID_ARG;
+    if (!aligned16(outs[x]) || (reinterpret_cast<uintptr_t>(lses[x]) & 3u)) return LITE_ERR_UNSUPPORTED;
+    mp.o[x] = static_cast<const __nv_bfloat16*>(outs[x]);
+    mp.lse[x] = lses[x];
+  }
+  mp.n = n_parts;
+  if (!aligned16(o) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))) return LITE_ERR_UNSUPPORTED;
   DeviceCache* dc = nullptr;
   if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
-  lite::AttnParams p = base_params(o, lse, B, H, N, d, scale, dc);
-  // every tile live, identity order, static striding over items (uniform cost): no scratch
-  return run_attention(dc, d, q, k, v, p, as_stream(stream));
+  const long long threads = static_cast<long long>(B) * H * N * (d / 8);
+  const long long want = (threads + 255) / 256;
+  // grid-stride; up to 8 resident 256-thread blocks per SM
+  const int blocks = int(std::min<long long>(want, static_cast<long long>(dc->sms) * 8));
+  cudaStream_t s = as_stream(stream);
+  __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(o);
+  if (d == 64) {
+    if (n_parts <= 2) lite::lite_lse_merge_kernel<64, 2><<<blocks, 256, 0, s>>>(mp, ob, lse, B, H, N);
+    else if (n_parts <= 4) lite::lite_lse_merge_kernel<64, 4><<<blocks, 256, 0, s>>>(mp, ob, lse, B, H, N);
+    else lite::lite_lse_merge_kernel<64, 8><<<blocks, 256, 0, s>>>(mp, ob, lse, B, H, N);
+  } else {
+    if (n_parts <= 2) lite::lite_lse_merge_kernel<128, 2><<<blocks, 256, 0, s>>>(mp, ob, lse, B, H, N);
+    else if (n_parts <= 4) lite::lite_lse_merge_kernel<128, 4><<<blocks, 256, 0, s>>>(mp, ob, lse, B, H, N);
+    else lite::lite_lse_merge_kernel<128, 8><<<blocks, 256, 0, s>>>(mp, ob, lse, B, H, N);
+  }
+  return cudaGetLastError() == cudaSuccess ? LITE_OK : LITE_ERR_CUDA;
 }
 
 #ifdef LITE_ATTN_TRACE
@@ -384,49 +519,13 @@ void* noalloc_scratch() {
 extern "C" int lite_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                                      const uint32_t* mask_in, uint32_t* mask_out, int B, int H, int N, int d,
                                      float scale, float tau, lite_stream_t stream) {
-  int st = check_qkvo(q, k, v, o, lse);
+  const FwdArgs a{q, k, v, o, lse, mask_in, mask_out, B, H, N, N, d, scale, tau};
+  const int st = validate_fwd(a);
   if (st) return st;
-  st = check_shapes(B, H, N, d);
-  if (st) return st;
-  if (std::isnan(tau)) return LITE_ERR_INVALID_ARG;
-  if (tau > 0.f && !debug_env()) return LITE_ERR_INVALID_ARG;
-  if ((mask_in && (reinterpret_cast<uintptr_t>(mask_in) & 3u)) || (mask_out && (reinterpret_cast<uintptr_t>(mask_out) & 3u)))
-    return LITE_ERR_UNSUPPORTED;
-  if (static_cast<long long>(B) * H > 8192) return LITE_ERR_UNSUPPORTED;
-
-  const int t = tile_for(d);
-  const int T = (N + t - 1) / t;
-  const size_t rows = size_t(B) * H * T;
-  const size_t list_b = align256(rows * T * sizeof(int16_t));
-  const size_t cnt_b = align256(rows * sizeof(int32_t));
-  const size_t need = list_b + 2 * cnt_b + 256;
-  if (need > LITE_NOALLOC_SCRATCH_BYTES) return LITE_ERR_SCRATCH_LIMIT;
-
+  if (fwd_scratch(a).total > LITE_NOALLOC_SCRATCH_BYTES) return LITE_ERR_SCRATCH_LIMIT;
   DeviceCache* dc = nullptr;
   if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
   char* base = static_cast<char*>(noalloc_scratch());
   if (!base) return LITE_ERR_CUDA;
-  cudaStream_t s = as_stream(stream);
-  lite::AttnParams p = base_params(o, lse, B, H, N, d, scale, dc);
-  const int W = p.W;
-  int16_t* list = reinterpret_cast<int16_t*>(base);
-  int32_t* counts = reinterpret_cast<int32_t*>(base + list_b);
-  int32_t* order = reinterpret_cast<int32_t*>(base + list_b + cnt_b);
-  int32_t* counter = reinterpret_cast<int32_t*>(base + list_b + 2 * cnt_b);
-
-  // the array keeps the previous call's contents: the work counter must start at zero
-  if (cudaMemsetAsync(counter, 0, sizeof(int32_t), s) != cudaSuccess) return LITE_ERR_CUDA;
-  lite::lite_compact_kernel<<<(int(rows) + 7) / 8, 256, 0, s>>>(mask_in, mask_out, list, counts, int(rows), T, W);
-  if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
-  const size_t sm = size_t(B * H + T) * sizeof(int32_t);
-  lite::lite_schedule_kernel<<<B * H, 512, sm, s>>>(counts, order, B * H, T);
-  if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
-  p.mask_out = mask_out;
-  p.list = list;
-  p.counts = counts;
-  p.order = order;
-  p.work_counter = counter;
-  p.tau_log2 = tau * 1.4426950408889634f;
-  p.skip_test = (mask_out != nullptr && tau > -INFINITY) ? 1 : 0;
-  return run_attention(dc, d, q, k, v, p, s);
+  return enqueue_fwd(dc, a, nullptr, base, as_stream(stream));
 }

@@ -4,7 +4,9 @@
 //    read one 32-bit word at a time from the top word down; lane l owns key tile 32*w + 31 - l, so a
 //    ballot plus a prefix popcount gives every live tile its slot in descending order (the README's
 //    reverse iteration order). The same pass copies the row into mask_out (with bits >= T cleared),
-//    which is where the attention kernel later ORs new flags.
+//    which is where the attention kernel later ORs new flags. With must-do / must-skip ranges the
+//    live set is (not masked or must-do) and not (must-skip and not must-do); must-do entries are
+//    tagged so that the attention kernel never flags them. The copied mask is mask_in unchanged.
 //  * lite_schedule_kernel: one CTA per head. Ranks the head among all heads by total live work,
 //    then places each of its query tiles by (live count desc, index asc) with an O(T^2) rank count
 //    in shared memory -- deterministic, no atomics on the output.
@@ -12,13 +14,23 @@
 
 #include <stdint.h>
 
+#include "attn_kernel.cuh"
+
 namespace lite {
 
+// Key tiles pinned by must-do / must-skip token ranges (README, must_do_list / must_skip_list),
+// as bitmaps in the Skip-Mask's word layout. Passed by value: Tk <= 4096 gives at most 128 words.
+struct RangeBits {
+  uint32_t live[128];  // must-do: always live, never flagged
+  uint32_t skip[128];  // must-skip (must-do already removed): always skipped
+};
+
 // mask_in may alias mask_out (in-place update): each warp reads a word before it writes it back.
-__global__ void __launch_bounds__(256) lite_compact_kernel(const uint32_t* mask_in,
-                                                          uint32_t* mask_out, int16_t* __restrict__ list,
-                                                          int32_t* __restrict__ counts, int rows, int T,
-                                                          int W) {
+// kRanges: apply RangeBits (live wins over skip and over the mask; tagged entries are never flagged).
+template <bool kRanges>
+__global__ void __launch_bounds__(256) lite_compact_kernel(const uint32_t* mask_in, uint32_t* mask_out,
+                                                          int16_t* __restrict__ list, int32_t* __restrict__ counts,
+                                                          int rows, int T, int W, const RangeBits ranges) {
   const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp_global >= rows) return;
@@ -29,10 +41,18 @@ __global__ void __launch_bounds__(256) lite_compact_kernel(const uint32_t* mask_
     uint32_t word = mask_in ? mask_in[row * W + w] : 0u;
     if (w == W - 1) word &= tail_mask;  // bits >= T carry no tile
     if (mask_out && lane == 0) mask_out[row * W + w] = word;
+    uint32_t forced = 0u;
+    if constexpr (kRanges) {
+      forced = ranges.live[w];
+      word = (word | ranges.skip[w]) & ~forced;
+    }
     const int j = w * 32 + 31 - lane;
     const bool live = (j < T) && !((word >> (31 - lane)) & 1u);
     const uint32_t bal = __ballot_sync(0xffffffffu, live);
-    if (live && list) list[row * T + count + __popc(bal & ((1u << lane) - 1u))] = int16_t(j);
+    if (live && list) {
+      const int tag = ((forced >> (31 - lane)) & 1u) ? kListNoFlag : 0;
+      list[row * T + count + __popc(bal & ((1u << lane) - 1u))] = int16_t(j | tag);
+    }
     count += __popc(bal);
   }
   if (lane == 0) counts[row] = count;

@@ -45,7 +45,11 @@ SIGNATURES = {
     "lite_set_option": ([_I, ctypes.c_longlong], _I),
     "lite_set_kernel_events": ([_P, _P], _I),
     "lite_attn_fwd_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _F, _P], _I),
+    "lite_attn_fwd_ex": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _F, _P], _I),
+    "lite_attn_dense_ex": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P], _I),
+    "lite_lse_merge": ([_P, _P, _I, _P, _P, _I, _I, _I, _I, _P], _I),
 }
+MAX_MERGE_PARTS = 8
 
 _lib = None
 
@@ -98,17 +102,37 @@ def lite_mask_geometry(N: int, d: int) -> Tuple[int, int, int]:
     return tile.value, T.value, W.value
 
 
+def _check_bf16(name, t):
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+        raise ValueError(f"{name} must be a contiguous 4-D bf16 CUDA tensor [B, N, H, d]")
+
+
 def _check_qkv(q, k, v):
     for name, t in (("q", q), ("k", k), ("v", v)):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
-            raise ValueError(f"{name} must be a contiguous 4-D bf16 CUDA tensor [B, N, H, d]")
+        _check_bf16(name, t)
     if not (q.shape == k.shape == v.shape):
         raise ValueError("q, k, v must have the same shape [B, N, H, d]")
 
 
-def new_mask(B: int, H: int, N: int, d: int, device=None) -> torch.Tensor:
-    """A fresh (all-live) Skip-Mask, int32 [B, H, T, W] holding uint32 bit patterns."""
-    _, T, W = lite_mask_geometry(N, d)
+def _check_qkv_cross(q, k, v):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_bf16(name, t)
+    if k.shape != v.shape or q.shape[0] != k.shape[0] or q.shape[2:] != k.shape[2:]:
+        raise ValueError("q [B, Nq, H, d] and k, v [B, Nk, H, d] must agree in B, H and d")
+
+
+def _ranges(r, name):
+    """README-style range list -> (ctypes int32 array or None, length)."""
+    if r is None or len(r) == 0:
+        return None, 0
+    vals = [int(x) for x in r]
+    return (ctypes.c_int32 * len(vals))(*vals), len(vals)
+
+
+def new_mask(B: int, H: int, N: int, d: int, device=None, Nk: Optional[int] = None) -> torch.Tensor:
+    """A fresh (all-live) Skip-Mask, int32 [B, H, Tq, Wk] holding uint32 bit patterns (Nk defaults to N)."""
+    _, T, _ = lite_mask_geometry(N, d)
+    _, _, W = lite_mask_geometry(N if Nk is None else Nk, d)
     return torch.zeros((B, H, T, W), dtype=torch.int32, device=device or "cuda")
 
 
@@ -123,9 +147,7 @@ def lite_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask_in: Op
         o = torch.empty_like(q)
     if lse is None and return_lse:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    for m in (mask_in, mask_out):
-        if m is not None and (m.dtype != torch.int32 or not m.is_contiguous() or not m.is_cuda):
-            raise ValueError("masks must be contiguous int32 CUDA tensors [B, H, T, W]")
+    _check_masks(mask_in, mask_out)
     st = load().lite_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _ptr(lse), _ptr(mask_in),
                               _ptr(mask_out), B, H, N, d, float(scale or 0.0), float(tau), _stream_handle(stream))
     _check("lite_attn_fwd", st)
@@ -205,4 +227,78 @@ def lite_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: 
                                       _ptr(mask_in), _ptr(mask_out), B, H, N, d, float(scale or 0.0), float(tau),
                                       _stream_handle(stream))
     _check("lite_attn_fwd_noalloc", st)
+    return o, lse
+
+
+def _check_masks(*masks):
+    for m in masks:
+        if m is not None and (m.dtype != torch.int32 or not m.is_contiguous() or not m.is_cuda):
+            raise ValueError("masks must be contiguous int32 CUDA tensors [B, H, Tq, Wk]")
+
+
+def lite_attn_fwd_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask_in: Optional[torch.Tensor] = None,
+                     mask_out: Optional[torch.Tensor] = None, must_do=None, must_skip=None,
+                     scale: Optional[float] = None, tau: float = -10.0, o: Optional[torch.Tensor] = None,
+                     lse: Optional[torch.Tensor] = None, return_lse: bool = True, stream=None):
+    """Partial attention: q [B, Nq, H, d] against k, v [B, Nk, H, d], with README-style must-do /
+    must-skip key-token range lists (see include/lite_attn.h). Returns (o, lse or None)."""
+    _check_qkv_cross(q, k, v)
+    B, Nq, H, d = q.shape
+    Nk = k.shape[1]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _check_masks(mask_in, mask_out)
+    do_arr, n_do = _ranges(must_do, "must_do")
+    skip_arr, n_skip = _ranges(must_skip, "must_skip")
+    st = load().lite_attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _ptr(lse), _ptr(mask_in),
+                                 _ptr(mask_out), ctypes.cast(do_arr, _P) if do_arr is not None else None, n_do,
+                                 ctypes.cast(skip_arr, _P) if skip_arr is not None else None, n_skip, B, H, Nq, Nk, d,
+                                 float(scale or 0.0), float(tau), _stream_handle(stream))
+    _check("lite_attn_fwd_ex", st)
+    return o, lse
+
+
+def lite_attn_dense_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float] = None,
+                       o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, return_lse: bool = True,
+                       stream=None):
+    """No-skip partial attention, q [B, Nq, H, d] against k, v [B, Nk, H, d]. Returns (o, lse or None)."""
+    _check_qkv_cross(q, k, v)
+    B, Nq, H, d = q.shape
+    Nk = k.shape[1]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    st = load().lite_attn_dense_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _ptr(lse), B, H, Nq, Nk,
+                                   d, float(scale or 0.0), _stream_handle(stream))
+    _check("lite_attn_dense_ex", st)
+    return o, lse
+
+
+def lite_lse_merge(parts, o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                   return_lse: bool = True, stream=None):
+    """Combine partial attentions [(o_p [B, N, H, d] bf16, lse_p [B, H, N] fp32), ...] over disjoint
+    key sets into (o, lse). o / lse may be one of the parts' tensors (in place)."""
+    parts = list(parts)
+    if not 1 <= len(parts) <= MAX_MERGE_PARTS:
+        raise ValueError(f"1 to {MAX_MERGE_PARTS} parts")
+    o0 = parts[0][0]
+    B, N, H, d = o0.shape
+    for op, lp in parts:
+        _check_bf16("o_p", op)
+        if op.shape != o0.shape:
+            raise ValueError("all partial outputs must have one shape [B, N, H, d]")
+        if lp.dtype != torch.float32 or not lp.is_contiguous() or tuple(lp.shape) != (B, H, N):
+            raise ValueError("lse_p must be contiguous fp32 [B, H, N]")
+    if o is None:
+        o = torch.empty_like(o0)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=o0.device)
+    outs = (_P * len(parts))(*[op.data_ptr() for op, _ in parts])
+    lses = (_P * len(parts))(*[lp.data_ptr() for _, lp in parts])
+    st = load().lite_lse_merge(ctypes.cast(outs, _P), ctypes.cast(lses, _P), len(parts), o.data_ptr(), _ptr(lse),
+                               B, H, N, d, _stream_handle(stream))
+    _check("lite_lse_merge", st)
     return o, lse

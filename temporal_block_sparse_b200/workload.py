@@ -170,13 +170,15 @@ class Trajectory:
             self.advance()
 
 
-def random_mask(B: int, H: int, T: int, density: float, seed: int, device="cpu") -> torch.Tensor:
-    """A random skip mask [B, H, T, ceil(T/32)] int32 (uint32 bit patterns); bits >= T are zero."""
-    W = (T + 31) // 32
+def random_mask(B: int, H: int, T: int, density: float, seed: int, device="cpu", Tk=None) -> torch.Tensor:
+    """A random skip mask [B, H, T, ceil(Tk/32)] int32 (uint32 bit patterns) for T query tiles and
+    Tk key tiles (Tk = T by default); bits >= Tk are zero."""
+    Tk = T if Tk is None else Tk
+    W = (Tk + 31) // 32
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     bits = torch.rand((B, H, T, W * 32), generator=g) < density
-    bits[..., T:] = False
+    bits[..., Tk:] = False
     weights = (2 ** torch.arange(32, dtype=torch.int64))
     words = (bits.view(B, H, T, W, 32).to(torch.int64) * weights).sum(-1)
     words = torch.where(words >= 2 ** 31, words - 2 ** 32, words).to(torch.int32)

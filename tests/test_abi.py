@@ -26,7 +26,8 @@ def declared_functions():
 def test_header_declares_the_abi():
     names = declared_functions()
     for expected in ("lite_attn_fwd", "lite_attn_dense", "lite_mask_to_list", "lite_mask_geometry",
-                     "lite_get_device_status", "lite_status_string", "lite_schedule"):
+                     "lite_get_device_status", "lite_status_string", "lite_schedule", "lite_attn_fwd_ex",
+                     "lite_attn_dense_ex", "lite_lse_merge"):
         assert expected in names
 
 
@@ -124,3 +125,66 @@ def test_binding_refuses_without_library(tmp_path):
             la.load(str(tmp_path / "missing.so"))
     finally:
         la._lib = saved
+
+
+def _arr(vals):
+    return (ctypes.c_int32 * max(1, len(vals)))(*vals) if vals else None
+
+
+def _fwd_ex(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, mi=None, mo=None, do=None, skip=None, B=1, H=1, Nq=256,
+            Nk=384, d=128, scale=0.0, tau=-3.0, n_do=None, n_skip=None):
+    da, sa = _arr(do), _arr(skip)
+    nd = len(do or []) if n_do is None else n_do
+    ns = len(skip or []) if n_skip is None else n_skip
+    return la.load().lite_attn_fwd_ex(q, k, v, o, lse, mi, mo, ctypes.cast(da, ctypes.c_void_p) if da else None, nd,
+                                      ctypes.cast(sa, ctypes.c_void_p) if sa else None, ns, B, H, Nq, Nk, d, scale,
+                                      tau, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), la.LITE_ERR_INVALID_ARG),
+    (dict(Nq=0), la.LITE_ERR_INVALID_ARG),
+    (dict(Nk=0), la.LITE_ERR_INVALID_ARG),
+    (dict(Nk=4097 * 128), la.LITE_ERR_UNSUPPORTED),
+    (dict(Nq=4097 * 128), la.LITE_ERR_UNSUPPORTED),
+    (dict(d=32), la.LITE_ERR_UNSUPPORTED),
+    (dict(tau=float("nan")), la.LITE_ERR_INVALID_ARG),
+    # README range convention: strictly descending pairs, start inclusive, end exclusive
+    (dict(do=[80, 60, 45]), la.LITE_ERR_INVALID_ARG),              # odd length
+    (dict(do=[60, 80]), la.LITE_ERR_INVALID_ARG),                  # start below end
+    (dict(do=[80, 60, 60, 40]), la.LITE_ERR_INVALID_ARG),          # end_0 == start_1
+    (dict(do=[80, 60, 70, 40]), la.LITE_ERR_INVALID_ARG),          # overlapping, not descending
+    (dict(skip=[80, 40, 10, -2]), la.LITE_ERR_INVALID_ARG),        # end below -1
+    (dict(skip=[40, 40]), la.LITE_ERR_INVALID_ARG),                # empty pair
+    (dict(do=None, n_do=2), la.LITE_ERR_INVALID_ARG),              # count without a list
+    (dict(do=[80, 60], n_do=-2), la.LITE_ERR_INVALID_ARG),
+])
+def test_fwd_ex_argument_errors(kw, code):
+    assert _fwd_ex(**kw) == code
+
+
+def test_dense_ex_argument_errors():
+    lib = la.load()
+    assert lib.lite_attn_dense_ex(None, FAKE, FAKE, FAKE, None, 1, 1, 128, 64, 128, 0.0, None) == la.LITE_ERR_INVALID_ARG
+    assert lib.lite_attn_dense_ex(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 128, 0, 128, 0.0, None) == la.LITE_ERR_INVALID_ARG
+    assert lib.lite_attn_dense_ex(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 128, 64, 48, 0.0, None) == la.LITE_ERR_UNSUPPORTED
+
+
+def test_lse_merge_argument_errors():
+    lib = la.load()
+    P = ctypes.c_void_p
+
+    def ptrs(*xs):
+        return ctypes.cast((P * len(xs))(*xs), P)
+
+    two = ptrs(FAKE, FAKE)
+    assert lib.lite_lse_merge(None, two, 2, FAKE, None, 1, 1, 64, 128, None) == la.LITE_ERR_INVALID_ARG
+    assert lib.lite_lse_merge(two, two, 0, FAKE, None, 1, 1, 64, 128, None) == la.LITE_ERR_INVALID_ARG
+    assert lib.lite_lse_merge(ptrs(*[FAKE] * 9), ptrs(*[FAKE] * 9), 9, FAKE, None, 1, 1, 64, 128, None) == \
+        la.LITE_ERR_UNSUPPORTED
+    assert lib.lite_lse_merge(two, two, 2, None, None, 1, 1, 64, 128, None) == la.LITE_ERR_INVALID_ARG
+    assert lib.lite_lse_merge(two, ptrs(FAKE, None), 2, FAKE, None, 1, 1, 64, 128, None) == la.LITE_ERR_INVALID_ARG
+    assert lib.lite_lse_merge(ptrs(FAKE, FAKE + 8), two, 2, FAKE, None, 1, 1, 64, 128, None) == la.LITE_ERR_UNSUPPORTED
+    assert lib.lite_lse_merge(two, ptrs(FAKE, FAKE + 2), 2, FAKE, None, 1, 1, 64, 128, None) == la.LITE_ERR_UNSUPPORTED
+    assert lib.lite_lse_merge(two, two, 2, FAKE, None, 1, 1, 64, 96, None) == la.LITE_ERR_UNSUPPORTED
+    assert lib.lite_lse_merge(two, two, 2, FAKE, None, 0, 1, 64, 128, None) == la.LITE_ERR_INVALID_ARG
