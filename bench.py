@@ -52,7 +52,7 @@ def parse_args():
     ap.add_argument("--tau", type=float, default=None, help="fixed tau instead of the workload's schedule")
     ap.add_argument("--cpu-sample-tiles", type=int, default=24, help="query tiles per step (reference arm)")
     ap.add_argument("--heads", type=int, default=None, help="override H (a smaller layer, e.g. for profiling)")
-    ap.add_argument("--study", choices=["sweep", "stress"], default=None,
+    ap.add_argument("--study", choices=["sweep", "stress", "partial"], default=None,
                     help="threshold sweep (720p shape) or stress-workload report instead of the headline line")
     ap.add_argument("--study-steps", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
@@ -78,6 +78,16 @@ def measured_peaks():
             d = json.load(f)
         return d.get("bf16_tflops"), d.get("bf16_tflops_sustained"), "measured"
     return 1590.0, 1400.0, "fallback"
+
+
+def measured_hbm_gbs() -> float:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            v = json.load(f).get("hbm_gbs")
+        if v:
+            return float(v)
+    return 6650.0  # fallback copy bandwidth of this GPU type
 
 
 def stored_traffic(workload: str):
@@ -541,12 +551,83 @@ def _skipped_bound(q, k, mask_in, mask_out, tau, tiles):
     return {"flagged_tiles_checked": n, "max_p_over_exp_tau": worst_p, "max_rowmass_over_cols_exp_tau": worst_mass}
 
 
+def run_partial_study(args):
+    """The README's text + video split of full self-attention: t2t, t2v, v2t without skipping, v2v
+    with the Skip-Mask, the two LSE merges, against dense attention over all tokens. One JSON line."""
+    from temporal_block_sparse_b200 import lite_attn as la
+
+    base = wlmod.WORKLOADS["720p"]
+    text = 512
+    steps = args.study_steps or 6
+    tau = -3.0 if args.tau is None else args.tau
+    B, Nv, H, d = base.B, base.N, base.H, base.d
+    N = text + Nv
+    tile, Tv, Wv = la.lite_mask_geometry(Nv, d)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(4242)
+    qt, kt, vt = (torch.randn((B, text, H, d), generator=g, device="cuda").to(torch.bfloat16) for _ in range(3))
+    tr = wlmod.Trajectory(base, device="cuda")
+    hbm_peak = measured_hbm_gbs()
+
+    # dense attention over all N tokens, same layout, for the baseline time
+    qv, kv, vv = tr.current()
+    qa, ka, va = (torch.cat([a, b], dim=1).contiguous() for a, b in ((qt, qv), (kt, kv), (vt, vv)))
+    oa = torch.empty_like(qa)
+    la_ = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    la.lite_attn_dense(qa, ka, va, o=oa, lse=la_)
+    full_ms = _time_call(lambda: la.lite_attn_dense(qa, ka, va, o=oa, lse=la_), reps=3)
+    del qa, ka, va, oa, la_
+
+    m_in = torch.zeros((B, H, Tv, Wv), dtype=torch.int32, device="cuda")
+    m_out = torch.empty_like(m_in)
+    bufs = {name: (torch.empty((B, n, H, d), dtype=torch.bfloat16, device="cuda"),
+                   torch.empty((B, H, n), dtype=torch.float32, device="cuda"))
+            for name, n in (("t2t", text), ("t2v", text), ("v2t", Nv), ("v2v", Nv), ("text", text), ("video", Nv))}
+    per_step = []
+    for t in range(steps):
+        qv, kv, vv = tr.current()
+        pieces = {
+            "t2t": lambda: la.lite_attn_dense_ex(qt, kt, vt, o=bufs["t2t"][0], lse=bufs["t2t"][1]),
+            "t2v": lambda: la.lite_attn_dense_ex(qt, kv, vv, o=bufs["t2v"][0], lse=bufs["t2v"][1]),
+            "v2t": lambda: la.lite_attn_dense_ex(qv, kt, vt, o=bufs["v2t"][0], lse=bufs["v2t"][1]),
+            "v2v": lambda: la.lite_attn_fwd_ex(qv, kv, vv, m_in, m_out, tau=tau, o=bufs["v2v"][0],
+                                               lse=bufs["v2v"][1]),
+            "merge_text": lambda: la.lite_lse_merge([bufs["t2t"], bufs["t2v"]], o=bufs["text"][0],
+                                                    lse=bufs["text"][1]),
+            "merge_video": lambda: la.lite_lse_merge([bufs["v2t"], bufs["v2v"]], o=bufs["video"][0],
+                                                     lse=bufs["video"][1]),
+        }
+        rec = {"step": t, "skipped_v2v": skipped_fraction(m_in, Tv)}
+        for name, fn in pieces.items():
+            rec[name + "_ms"] = min(_time_call(fn), _time_call(fn))
+        rec["total_ms"] = sum(rec[n + "_ms"] for n in pieces)
+        rec["speedup_vs_full_dense"] = full_ms / rec["total_ms"]
+        per_step.append(rec)
+        m_in, m_out = m_out, m_in
+        tr.advance()
+    assert la.lite_get_device_status() == 0
+    # LSE merge kernel on the video rows: algorithmic bytes = rows * (2 parts + 1 output) * (2 d + 4)
+    rows = B * H * Nv
+    merge_bytes = rows * 3 * (2 * d + 4)
+    merge_ms = min(r["merge_video_ms"] for r in per_step)
+    achieved = merge_bytes / (merge_ms * 1e-3) / 1e9
+    line = {"study": "partial", "workload": f"text {text} + 720p video: B={B} H={H} Nv={Nv} d={d}", "tau": tau,
+            "steps": steps, "full_dense_ms": full_ms,
+            "merge_roofline": {"bound": "hbm", "bytes_per_launch": merge_bytes, "ms": merge_ms,
+                               "achieved_gbs": achieved, "peak_gbs": hbm_peak,
+                               "frac": achieved / hbm_peak if hbm_peak else None},
+            "per_step": per_step}
+    print(json.dumps(line), flush=True)
+
+
 def run_study(args):
     """Threshold sweep and stress reports (one JSON line per run; not the headline metric)."""
     from temporal_block_sparse_b200 import lite_attn as la
 
     torch.cuda.set_device(0)
     la.load()
+    if args.study == "partial":
+        return run_partial_study(args)
     if args.study == "sweep":
         base = wlmod.WORKLOADS["sweep"]
         steps = args.study_steps or base.steps

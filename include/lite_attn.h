@@ -255,7 +255,7 @@ int lite_attn_dense_ex(const void* q, const void* k, const void* v, void* o, flo
  *  n_parts       1 .. 8.
  *  o        out  device bf16 [B, N, H, d]; may be one of outs (in place).
  *  lse      out  device fp32 [B, H, N], or NULL; may be one of lses.
- *  B, H, N, d    d in {64, 128}.
+ *  B, H, N, d    d in {64, 128}; B*H*N*d/8 < 2^31 (LITE_ERR_UNSUPPORTED otherwise).
  * The two host arrays are read during the call only.
  */
 int lite_lse_merge(const void* const* outs, const float* const* lses, int n_parts, void* o,

@@ -2,6 +2,7 @@
 
 from __future__ import annotations
 
+import glob
 import os
 import shutil
 import subprocess
@@ -10,8 +11,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SOURCES = [os.path.join(HERE, "csrc", "lite_attn_api.cu")]
-DEPS = SOURCES + [os.path.join(HERE, "csrc", f) for f in ("attn_kernel.cuh", "mask_kernels.cuh", "sm100_ptx.cuh")] + [
-    os.path.join(ROOT, "include", "lite_attn.h")]
+DEPS = SOURCES + sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh"))) + [os.path.join(ROOT, "include", "lite_attn.h")]
 OUT = os.path.join(HERE, "liblite_attn.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

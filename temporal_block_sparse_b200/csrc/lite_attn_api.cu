@@ -457,6 +457,7 @@ int lite_lse_merge(const void* const* outs, const float* const* lses, int n_part
   }
   mp.n = n_parts;
   if (!aligned16(o) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))) return LITE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * N * (d / 8) >= (1ll << 31)) return LITE_ERR_UNSUPPORTED;
   DeviceCache* dc = nullptr;
   if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
   const long long threads = static_cast<long long>(B) * H * N * (d / 8);

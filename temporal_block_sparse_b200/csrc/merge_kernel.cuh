@@ -9,10 +9,11 @@
 // with lse -inf.
 //
 // HBM-bound: per row it reads P * (2 d + 4) bytes and writes 2 d + 4. Each thread owns 16 bytes
-// (8 bf16) of one row, so a row of d = 128 is 16 consecutive threads reading whole 32-byte sectors;
-// rows are walked in (b, h, n) order, which makes the lse reads of a warp contiguous too. All
-// parts' loads of a thread are issued before any arithmetic, so P * 16 bytes per thread are in
-// flight.
+// (8 bf16) of one row. Rows are walked in memory order of o, (b, n, h), so a warp reads and writes
+// one contiguous 512-byte stretch of every part (d = 128: two rows); the lse values it needs are
+// strided by N but few (24 MB for a 720p layer's two parts), and the n-neighbours that share their
+// sectors are processed right after, out of L2. All parts' loads of a thread are issued before any
+// arithmetic. Index arithmetic is 32-bit (the host refuses B*H*N*d/8 >= 2^31).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -36,28 +37,29 @@ template <int D, int MP>
 __global__ void __launch_bounds__(256) lite_lse_merge_kernel(const MergeParts parts, __nv_bfloat16* o, float* lse,
                                                              int B, int H, int N) {
   constexpr int G = D / 8;  // threads per row
-  const long long rows = static_cast<long long>(B) * H * N;
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  const uint32_t total = uint32_t(B) * H * N * G;
+  const uint32_t stride = gridDim.x * blockDim.x;
   // the loop bound is uniform over a warp (whole warps step together), so __syncwarp is legal
-  const long long warp_base0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) & ~31ll;
-  const int lane = threadIdx.x & 31;
-  for (long long base = warp_base0; base < rows * G; base += stride) {
-    const long long gid = base + lane;
-    const bool valid = gid < rows * G;
-    const long long row = valid ? gid / G : 0;  // (b * H + h) * N + n
-    const int g = int(gid - row * G);
-    const long long bh = row / N;
-    const int n = int(row - bh * N);
-    const int b = int(bh / H);
-    const int h = int(bh - static_cast<long long>(b) * H);
-    const size_t off = ((static_cast<size_t>(b) * N + n) * H + h) * D + size_t(g) * 8;
+  const uint32_t warp_base0 = (blockIdx.x * blockDim.x + threadIdx.x) & ~31u;
+  const uint32_t lane = threadIdx.x & 31;
+  for (uint32_t base = warp_base0; base < total; base += stride) {
+    const uint32_t gid = base + lane;
+    const bool valid = gid < total;
+    const uint32_t row = valid ? gid / G : 0;  // (b * N + n) * H + h: the memory order of o
+    const uint32_t g = gid - row * G;
+    const uint32_t bn = row / uint32_t(H);
+    const uint32_t h = row - bn * uint32_t(H);
+    const uint32_t b = bn / uint32_t(N);
+    const uint32_t n = bn - b * uint32_t(N);
+    const size_t off = size_t(row) * D + g * 8;
+    const size_t lrow = (size_t(b) * H + h) * N + n;
 
     float l[MP];
     uint4 v[MP];
 #pragma unroll
     for (int p = 0; p < MP; ++p) {
       if (p < parts.n && valid) {
-        l[p] = parts.lse[p][row];
+        l[p] = parts.lse[p][lrow];
         v[p] = *reinterpret_cast<const uint4*>(parts.o[p] + off);
       } else {
         l[p] = -INFINITY;
@@ -102,7 +104,7 @@ __global__ void __launch_bounds__(256) lite_lse_merge_kernel(const MergeParts pa
         r[e] = *reinterpret_cast<uint32_t*>(&h2);
       }
       *reinterpret_cast<uint4*>(o + off) = res;
-      if (lse && g == 0) lse[row] = out_lse;
+      if (lse && g == 0) lse[lrow] = out_lse;
     }
   }
 }
