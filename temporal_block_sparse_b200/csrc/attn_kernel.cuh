@@ -120,15 +120,18 @@ struct AttnCfg {
   static_assert(BN == 64 || BN == 128, "tile");
   static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  // one TMA box per tile writes its d/64 panels [rows][128 B] back to back
+  static_assert(NCHUNK == 1 || (Q_CHUNK == BQ * 128 && KV_CHUNK == BN * 128), "panel strides");
 };
 
 // Control block in shared memory (barriers are 8-byte mbarrier objects).
 struct alignas(8) AttnCtl {
   uint64_t q_full, q_empty;
   uint64_t k_full[2], v_full[3];     // K_t (stage t%2) / V_t (stage t%3) landed
-  uint64_t s_full[2], p_full[2];     // S_t ready / P_t written (buffer t%2, one warpgroup each)
+  uint64_t s_full[2];                // S_t ready (buffer t%2, one warpgroup each)
+  uint64_t p_lo[2], p_hi[2];         // first / second half of P_t's key columns written
   uint64_t pv_done[2];               // last PV of group g in an item finished (accumulator g)
-  uint64_t mx_full[4];               // row maxima of tile t posted in mailbox slot t%4
+  uint64_t mx_full[4], mx_empty[4];  // row maxima of tile t posted in / read from mailbox slot t%4
   uint64_t o_free;                   // epilogue has read both O accumulators
   uint64_t item_full[2], item_empty[2];
   uint64_t drain;
@@ -263,13 +266,17 @@ __global__ void __launch_bounds__(320, 1)
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(BAR(k_full[b]), 1);
       ptx::mbar_init(BAR(s_full[b]), 1);
-      ptx::mbar_init(BAR(p_full[b]), 128);
+      ptx::mbar_init(BAR(p_lo[b]), 128);
+      ptx::mbar_init(BAR(p_hi[b]), 128);
       ptx::mbar_init(BAR(pv_done[b]), 1);
       ptx::mbar_init(BAR(item_full[b]), 1);
       ptx::mbar_init(BAR(item_empty[b]), 9);  // MMA thread + one lane of each softmax warp
     }
     for (int b = 0; b < 3; ++b) ptx::mbar_init(BAR(v_full[b]), 1);
-    for (int b = 0; b < 4; ++b) ptx::mbar_init(BAR(mx_full[b]), 128);
+    for (int b = 0; b < 4; ++b) {
+      ptx::mbar_init(BAR(mx_full[b]), 128);
+      ptx::mbar_init(BAR(mx_empty[b]), 128);
+    }
     ptx::mbar_init(BAR(o_free), 256);
     ptx::mbar_init(BAR(drain), 1);
     ctl->abort = 0;
@@ -325,8 +332,7 @@ __global__ void __launch_bounds__(320, 1)
         if (qn >= 1) ok = wt.wait(BAR(q_empty), (qn - 1) & 1);
         if (!ok) break;
         ptx::mbar_arrive_expect_tx(BAR(q_full), C::Q_TX);
-        for (int c = 0; c < C::NCHUNK; ++c)
-          ptx::tma_load_4d(sQ + c * C::Q_CHUNK, &tmQ, BAR(q_full), c * 64, it.h, it.qi * C::BQ, it.b);
+        ptx::tma_load_5d(sQ, &tmQ, BAR(q_full), 0, it.qi * C::BQ, 0, it.h, it.b);
         q_armed = true;
         q_par = qn & 1;
         ++qn;
@@ -340,9 +346,7 @@ __global__ void __launch_bounds__(320, 1)
           if (t >= 2) ok = wt.wait(BAR(s_full[t & 1]), ((t - 2) >> 1) & 1);
           if (!ok) break;
           ptx::mbar_arrive_expect_tx(BAR(k_full[t & 1]), C::KV_TX);
-          for (int c = 0; c < C::NCHUNK; ++c)
-            ptx::tma_load_4d(sK + (t & 1) * C::KV_BYTES + c * C::KV_CHUNK, &tmK, BAR(k_full[t & 1]), c * 64, it.h,
-                             j * BN, it.b);
+          ptx::tma_load_5d(sK + (t & 1) * C::KV_BYTES, &tmK, BAR(k_full[t & 1]), 0, j * BN, 0, it.h, it.b);
           LITE_TRACE(0, 1, t);
           k_armed[t & 1] = true;
           k_par[t & 1] = (t >> 1) & 1;
@@ -350,9 +354,7 @@ __global__ void __launch_bounds__(320, 1)
           if (t >= 3) ok = wt.wait(BAR(s_full[(t - 1) & 1]), ((t - 1) >> 1) & 1);
           if (!ok) break;
           ptx::mbar_arrive_expect_tx(BAR(v_full[vs]), C::KV_TX);
-          for (int c = 0; c < C::NCHUNK; ++c)
-            ptx::tma_load_4d(sV + vs * C::KV_BYTES + c * C::KV_CHUNK, &tmV, BAR(v_full[vs]), c * 64, it.h, j * BN,
-                             it.b);
+          ptx::tma_load_5d(sV + vs * C::KV_BYTES, &tmV, BAR(v_full[vs]), 0, j * BN, 0, it.h, it.b);
           LITE_TRACE(0, 3, t);
           v_armed[vs] = true;
           v_par[vs] = (t / 3) & 1;
@@ -431,7 +433,7 @@ __global__ void __launch_bounds__(320, 1)
             const uint32_t t = t0 + pv;
             if (pv == 0 && qn >= 1 && !wt.wait(BAR(o_free), (qn - 1) & 1)) { ok = false; break; }
             LITE_TRACE(1, 3, t);
-            if (!wt.wait(BAR(p_full[t & 1]), (t >> 1) & 1)) { ok = false; break; }
+            if (!wt.wait(BAR(p_lo[t & 1]), (t >> 1) & 1)) { ok = false; break; }
             LITE_TRACE(1, 4, t);
             if (!wt.wait(BAR(v_full[t % 3]), (t / 3) & 1)) { ok = false; break; }
             LITE_TRACE(1, 5, t);
@@ -439,10 +441,18 @@ __global__ void __launch_bounds__(320, 1)
             const uint32_t p_tmem = tmem + C::S_COL + (t & 1) * BN;
             const uint32_t o_tmem = tmem + C::O_COL + (t & 1) * D;
             const uint64_t vd = v_desc0 + uint64_t(((t % 3) * C::KV_BYTES) >> 4);
+            // the first half of the key columns starts as soon as its P is written; the softmax
+            // computes the second half meanwhile
 #pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk)
+            for (int kk = 0; kk < BN / 32; ++kk)
               ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + uint64_t(kk * 128), C::IDESC_PV,
                           (pv < 2 && kk == 0) ? 0u : 1u);
+            if (!wt.wait(BAR(p_hi[t & 1]), (t >> 1) & 1)) { ok = false; break; }
+            LITE_TRACE(1, 7, t);
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int kk = BN / 32; kk < BN / 16; ++kk)
+              ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + uint64_t(kk * 128), C::IDESC_PV, 1u);
             // the epilogue of group t%2 waits for the last PV into its accumulator
             if (pv >= it.n - 2) ptx::mma_commit(BAR(pv_done[t & 1]));
             LITE_TRACE(1, 6, t);
@@ -500,6 +510,7 @@ __global__ void __launch_bounds__(320, 1)
         __syncwarp();
         ptx::tc_fence_after();
         const uint32_t s_tmem = tmem + lane_base + C::S_COL + grp * BN;
+        // the whole S row is read once and stays in registers for the max and the exponentials
         uint32_t sr[BN];
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c)
@@ -525,27 +536,16 @@ __global__ void __launch_bounds__(320, 1)
           m3 = ptx::fmax3(m3, s[x + 6], s[x + 7]);
         }
         const float loc = ptx::fmax3(m0, m1, fmaxf(m2, m3)) * p.scale_log2;
-        // post this tile's row maxima for the other group, then fold in the previous tile's
         if (r == 0) LITE_TRACE(2 + grp, 2, t);
+        // post this tile's row maxima for the group that takes tile t+1 (they enter its QK-Skip
+        // running max). Slot t%4 is refilled every four tiles, after its reader took tile t-4's.
+        if (t >= 4) wt.wait(BAR(mx_empty[t & 3]), ((t >> 2) - 1) & 1);
         mailbox[(t & 3) * 128 + r] = loc;
         ptx::mbar_arrive(BAR(mx_full[t & 3]));
-        if (idx > 0) {
-          wt.wait(BAR(mx_full[(t - 1) & 3]), ((t - 1) >> 2) & 1);
-          m_true = fmaxf(m_true, mailbox[((t - 1) & 3) * 128 + r]);
-        }
-        if (r == 0) LITE_TRACE(2 + grp, 3, t);
-        if (p.skip_test) {
-          // QK-Skip: flag tile j when loc - m < tau for every valid row (m over earlier tiles)
-          const bool pred = !valid_row || (loc - m_true < p.tau_log2);
-          const bool flag = ptx::named_bar_and(vote_bar, 128, pred);
-          if (flag && may_flag && r == 0 && p.mask_out && !ctl->abort)
-            atomicOr(p.mask_out + size_t(it.row) * p.W + (j >> 5), 1u << (j & 31));
-        }
-        if (r == 0) LITE_TRACE(2 + grp, 4, t);
-        m_true = fmaxf(m_true, loc);
         // lazy rescale of this group's accumulator: move the reference only when the tile max
         // exceeds it by more than 8 (log2 units). The previous PV into this accumulator (tile t-2)
-        // was issued before QK_t, so it has completed now that S_t is ready.
+        // was issued before QK_t, so it has completed now that S_t is ready; the rescaled O is
+        // stored before any P of this tile is released to the MMA thread.
         const bool need = loc > m_used + 8.0f;
         float alpha = 1.f;
         if (need) {
@@ -553,51 +553,7 @@ __global__ void __launch_bounds__(320, 1)
           m_used = loc;
           l *= alpha;
         }
-        const bool warp_need = __any_sync(0xffffffffu, need) && (idx >= 2);
-        // P = 2^(s*scale*log2e - m_used) as bf16 pairs, written over S columns already read: the
-        // chunk loop re-reads S 32 columns at a time (compact code, few live registers) and chunk
-        // c's P lands in columns [16c, 16c+16), all read by chunks <= c. Packed fp32x2 arithmetic
-        // for the affine step and the row sum; one column pair in four is exponentiated on the FMA
-        // pipe, the rest on MUFU, to balance the two units and the issue slots.
-        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-        const float2 nm2 = make_float2(-m_used, -m_used);
-        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        // one chunk of 32 S columns -> 16 bf16 pairs of P at column 16c
-        auto exp_chunk = [&](const uint32_t (&q)[32], int c) {
-          const int vc = valid_cols - c * 32;  // valid columns in this chunk (>= 32 except in the tail)
-          uint32_t pk[16];
-#pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            float s0 = __uint_as_float(q[2 * x]), s1 = __uint_as_float(q[2 * x + 1]);
-            if (vc < 32) {
-              s0 = 2 * x < vc ? s0 : -INFINITY;
-              s1 = 2 * x + 1 < vc ? s1 : -INFINITY;
-            }
-            const float2 a = __ffma2_rn(make_float2(s0, s1), sc2, nm2);
-            const float2 pp = ((x & 3) == 3) ? exp2_poly2(a) : make_float2(ptx::ex2(a.x), ptx::ex2(a.y));
-            acc[x & 3] = __fadd2_rn(acc[x & 3], pp);
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(pp.x, pp.y);
-            pk[x] = *reinterpret_cast<uint32_t*>(&h2);
-          }
-          ptx::tmem_st16(s_tmem + c * 16, pk);
-        };
-        // double-buffered: the next chunk's TMEM load is in flight while this chunk is computed
-        // (tcgen05.wait::ld waits for all of this thread's loads, so the next load is issued after it)
-        uint32_t qa[32], qb[32];
-        ptx::tmem_ld32(s_tmem, qa);
-        ptx::tmem_wait_ld();
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; c += 2) {
-          ptx::tmem_ld32(s_tmem + (c + 1) * 32, qb);
-          exp_chunk(qa, c);
-          ptx::tmem_wait_ld();
-          if (c + 2 < BN / 32) ptx::tmem_ld32(s_tmem + (c + 2) * 32, qa);
-          exp_chunk(qb, c + 1);
-          ptx::tmem_wait_ld();
-        }
-        const float2 acc2 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-        l += acc2.x + acc2.y;
-        if (warp_need) {
+        if (__any_sync(0xffffffffu, need) && idx >= 2) {
           const uint32_t o_tmem = tmem + lane_base + C::O_COL + grp * D;
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
@@ -609,10 +565,56 @@ __global__ void __launch_bounds__(320, 1)
             ptx::tmem_st32(o_tmem + c * 32, rr);
           }
         }
-        ptx::tmem_wait_st();
+        // P = 2^(s*scale*log2e - m_used) as bf16 pairs over the S columns (chunk c of 32 key
+        // columns -> TMEM columns [16c, 16c+16)), released in two halves of the key columns so
+        // that the first half of PV runs while the second half is exponentiated. Packed fp32x2
+        // arithmetic for the affine step and the row sum; one column pair in four is exponentiated
+        // on the FMA pipe, the rest on MUFU.
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 nm2 = make_float2(-m_used, -m_used);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+          for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+              const float2 a = __ffma2_rn(make_float2(s[32 * c + 2 * x], s[32 * c + 2 * x + 1]), sc2, nm2);
+              const float2 pp = ((x & 3) == 3) ? exp2_poly2(a) : make_float2(ptx::ex2(a.x), ptx::ex2(a.y));
+              acc[x & 3] = __fadd2_rn(acc[x & 3], pp);
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(pp.x, pp.y);
+              pk[x] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            ptx::tmem_st16(s_tmem + c * 16, pk);
+          }
+          ptx::tmem_wait_st();
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(half == 0 ? BAR(p_lo[grp]) : BAR(p_hi[grp]));
+          if (half == 0 && r == 0) LITE_TRACE(2 + grp, 5, t);
+        }
         if (r == 0) LITE_TRACE(2 + grp, 6, t);
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(BAR(p_full[grp]));
+        const float2 acc2 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+        l += acc2.x + acc2.y;
+        // QK-Skip vote, off the path from S to P. The running max over the tiles visited before t
+        // takes in tile t-1's maxima from the other group; every posted slot is consumed (also at
+        // the first tile of an item, where the value is not used) so that the slots stay in step.
+        if (t >= 1) {
+          wt.wait(BAR(mx_full[(t - 1) & 3]), ((t - 1) >> 2) & 1);
+          const float prev = mailbox[((t - 1) & 3) * 128 + r];
+          ptx::mbar_arrive(BAR(mx_empty[(t - 1) & 3]));
+          if (idx > 0) m_true = fmaxf(m_true, prev);
+        }
+        if (r == 0) LITE_TRACE(2 + grp, 3, t);
+        if (p.skip_test) {
+          // QK-Skip: flag tile j when loc - m < tau for every valid row (m over earlier tiles)
+          const bool pred = !valid_row || (loc - m_true < p.tau_log2);
+          const bool flag = ptx::named_bar_and(vote_bar, 128, pred);
+          if (flag && may_flag && r == 0 && p.mask_out && !ctl->abort)
+            atomicOr(p.mask_out + size_t(it.row) * p.W + (j >> 5), 1u << (j & 31));
+        }
+        if (r == 0) LITE_TRACE(2 + grp, 4, t);
+        m_true = fmaxf(m_true, loc);
       }
       // epilogue: each group waits for its last PV, the two partial softmaxes are combined,
       // group g stores columns [g*D/2, (g+1)*D/2) of O (bf16) and group 0 the lse

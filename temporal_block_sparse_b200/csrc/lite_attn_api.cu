@@ -115,13 +115,16 @@ int check_qkvo(const void* q, const void* k, const void* v, const void* o, const
   return LITE_OK;
 }
 
-// [B, N, H, d] bf16 viewed as a 4-D tensor (d, H, N, B); box = 64 elements x 1 head x rows x 1.
+// [B, N, H, d] bf16 viewed as a 5-D tensor (64, N, d/64, H, B): the head dim is split into 64-element
+// (128-byte) chunks and the chunk index is placed OUTSIDE the token index, so that one box of
+// 64 x rows x d/64 lands in shared memory as d/64 consecutive [rows][128 B] swizzle-128B panels --
+// the K-major operand layout of the MMA -- in a single TMA request per tile.
 bool make_tmap(CUtensorMap* map, const void* ptr, int B, int N, int H, int d, int rows) {
-  cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(H), cuuint64_t(N), cuuint64_t(B)};
-  cuuint64_t strides[3] = {cuuint64_t(d) * 2, cuuint64_t(H) * d * 2, cuuint64_t(N) * H * d * 2};
-  cuuint32_t box[4] = {64, 1, cuuint32_t(rows), 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+  cuuint64_t dims[5] = {64, cuuint64_t(N), cuuint64_t(d / 64), cuuint64_t(H), cuuint64_t(B)};
+  cuuint64_t strides[4] = {cuuint64_t(H) * d * 2, 128, cuuint64_t(d) * 2, cuuint64_t(N) * H * d * 2};
+  cuuint32_t box[5] = {64, cuuint32_t(rows), cuuint32_t(d / 64), 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
