@@ -261,6 +261,25 @@ int lite_attn_dense_ex(const void* q, const void* k, const void* v, void* o, flo
 int lite_lse_merge(const void* const* outs, const float* const* lses, int n_parts, void* o,
                    float* lse, int B, int H, int N, int d, lite_stream_t stream);
 
+/*
+ * lite_dropped_mass -- the error a Skip-Mask introduces at one step, for the accumulated-error
+ * calibration of the QK-Skip threshold ("Lite Attention Temporal Sparse" skill page, Architecture
+ * Overview: Accumulated-Error Calibration; README contribution list, "Error Calibration").
+ *
+ * For every (b, h) and query row n, the softmax probability that the skipped key tiles hold under
+ * the dense softmax: 1 - exp(lse_live - lse_full), computed as -expm1 in fp32 and clamped to [0, 1];
+ * a row whose lse_live is -inf (no live tile) drops 1.
+ *
+ *  lse_live  in   device fp32 [B, H, N]: lse of lite_attn_fwd with the mask as mask_in (tau = -inf).
+ *  lse_full  in   device fp32 [B, H, N]: lse of lite_attn_dense on the same q, k, v.
+ *  row_mass  out  device fp32 [B, H, N], or NULL.
+ *  stats     out  device fp32 [2]: {largest per-row value, sum over all rows}. The call zeroes it
+ *                 on `stream` first; read it after the stream has reached this call.
+ *  Pointers must be 4-byte aligned (16-byte alignment of all three arrays enables vector loads).
+ */
+int lite_dropped_mass(const float* lse_live, const float* lse_full, float* row_mass, float* stats,
+                      int B, int H, int N, lite_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

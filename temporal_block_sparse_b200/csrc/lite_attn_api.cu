@@ -15,6 +15,7 @@
 #include <mutex>
 
 #include "attn_kernel.cuh"
+#include "calib_kernels.cuh"
 #include "lite_attn.h"
 #include "mask_kernels.cuh"
 #include "merge_kernel.cuh"
@@ -478,6 +479,23 @@ int lite_lse_merge(const void* const* outs, const float* const* lses, int n_part
     else if (n_parts <= 4) lite::lite_lse_merge_kernel<128, 4><<<blocks, 256, 0, s>>>(mp, ob, lse, B, H, N);
     else lite::lite_lse_merge_kernel<128, 8><<<blocks, 256, 0, s>>>(mp, ob, lse, B, H, N);
   }
+  return cudaGetLastError() == cudaSuccess ? LITE_OK : LITE_ERR_CUDA;
+}
+
+int lite_dropped_mass(const float* lse_live, const float* lse_full, float* row_mass, float* stats, int B, int H,
+                      int N, lite_stream_t stream) {
+  if (!lse_live || !lse_full || !stats || B <= 0 || H <= 0 || N <= 0) return LITE_ERR_INVALID_ARG;
+  const uintptr_t mis = reinterpret_cast<uintptr_t>(lse_live) | reinterpret_cast<uintptr_t>(lse_full) |
+                        reinterpret_cast<uintptr_t>(row_mass) | reinterpret_cast<uintptr_t>(stats);
+  if (mis & 3u) return LITE_ERR_UNSUPPORTED;
+  DeviceCache* dc = nullptr;
+  if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  const long long rows = static_cast<long long>(B) * H * N;
+  if (cudaMemsetAsync(stats, 0, 2 * sizeof(float), s) != cudaSuccess) return LITE_ERR_CUDA;
+  const long long want = (rows + 1023) / 1024;  // 4 rows per thread, 256 threads per block
+  const int blocks = int(std::max<long long>(1, std::min<long long>(want, static_cast<long long>(dc->sms) * 8)));
+  lite::lite_dropped_mass_kernel<<<blocks, 256, 0, s>>>(lse_live, lse_full, row_mass, stats, rows);
   return cudaGetLastError() == cudaSuccess ? LITE_OK : LITE_ERR_CUDA;
 }
 

@@ -48,6 +48,7 @@ SIGNATURES = {
     "lite_attn_fwd_ex": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _F, _P], _I),
     "lite_attn_dense_ex": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P], _I),
     "lite_lse_merge": ([_P, _P, _I, _P, _P, _I, _I, _I, _I, _P], _I),
+    "lite_dropped_mass": ([_P, _P, _P, _P, _I, _I, _I, _P], _I),
 }
 MAX_MERGE_PARTS = 8
 
@@ -302,3 +303,24 @@ def lite_lse_merge(parts, o: Optional[torch.Tensor] = None, lse: Optional[torch.
                                B, H, N, d, _stream_handle(stream))
     _check("lite_lse_merge", st)
     return o, lse
+
+
+def lite_dropped_mass(lse_live: torch.Tensor, lse_full: torch.Tensor, row_mass: Optional[torch.Tensor] = None,
+                      stats: Optional[torch.Tensor] = None, stream=None):
+    """Per-row softmax mass a Skip-Mask drops, 1 - exp(lse_live - lse_full), for lse tensors
+    [B, H, N] fp32 on the GPU. Returns (row_mass or None, stats) with stats a device fp32 [2] tensor
+    {largest per-row value, sum over rows}; reading it synchronises."""
+    for name, t in (("lse_live", lse_live), ("lse_full", lse_full)):
+        if t.dtype != torch.float32 or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError(f"{name} must be a contiguous fp32 [B, H, N] tensor")
+    if lse_live.shape != lse_full.shape:
+        raise ValueError("lse_live and lse_full differ in shape")
+    B, H, N = lse_live.shape
+    if row_mass is not None and (row_mass.shape != lse_live.shape or row_mass.dtype != torch.float32):
+        raise ValueError("row_mass must match the lse tensors")
+    if stats is None:
+        stats = torch.empty(2, dtype=torch.float32, device=lse_live.device)
+    st = load().lite_dropped_mass(lse_live.data_ptr(), lse_full.data_ptr(), _ptr(row_mass), stats.data_ptr(), B, H,
+                                  N, _stream_handle(stream))
+    _check("lite_dropped_mass", st)
+    return row_mass, stats

@@ -27,7 +27,7 @@ def test_header_declares_the_abi():
     names = declared_functions()
     for expected in ("lite_attn_fwd", "lite_attn_dense", "lite_mask_to_list", "lite_mask_geometry",
                      "lite_get_device_status", "lite_status_string", "lite_schedule", "lite_attn_fwd_ex",
-                     "lite_attn_dense_ex", "lite_lse_merge"):
+                     "lite_attn_dense_ex", "lite_lse_merge", "lite_dropped_mass"):
         assert expected in names
 
 
@@ -188,3 +188,14 @@ def test_lse_merge_argument_errors():
     assert lib.lite_lse_merge(two, ptrs(FAKE, FAKE + 2), 2, FAKE, None, 1, 1, 64, 128, None) == la.LITE_ERR_UNSUPPORTED
     assert lib.lite_lse_merge(two, two, 2, FAKE, None, 1, 1, 64, 96, None) == la.LITE_ERR_UNSUPPORTED
     assert lib.lite_lse_merge(two, two, 2, FAKE, None, 0, 1, 64, 128, None) == la.LITE_ERR_INVALID_ARG
+
+
+def test_dropped_mass_argument_checks():
+    lib = la.load()
+    f = lib.lite_dropped_mass
+    assert f(None, FAKE, None, FAKE, 1, 1, 8, None) == la.LITE_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, None, None, 1, 1, 8, None) == la.LITE_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, None, FAKE, 0, 1, 8, None) == la.LITE_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, None, FAKE, 1, 1, -3, None) == la.LITE_ERR_INVALID_ARG
+    assert f(FAKE + 2, FAKE, None, FAKE, 1, 1, 8, None) == la.LITE_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE + 1, FAKE, 1, 1, 8, None) == la.LITE_ERR_UNSUPPORTED
