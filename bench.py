@@ -761,6 +761,15 @@ def run_study(args):
                 rec["compaction_ms"] = _time_call(lambda: lib.lite_mask_to_list(m_in.data_ptr(), lst.data_ptr(),
                                                                                 cnt.data_ptr(), B, H, N, d, sh))
                 rec["schedule_ms"] = _time_call(lambda: lib.lite_schedule(cnt.data_ptr(), ordr.data_ptr(), B, H, T, sh))
+                # range-encoded Skip-List of the same mask: time and bytes written against the per-tile list
+                rng = torch.empty((B, H, T, T + 1), dtype=torch.int16, device="cuda")
+                nrun = torch.empty((B, H, T), dtype=torch.int32, device="cuda")
+                rec["ranges_ms"] = _time_call(lambda: lib.lite_mask_to_ranges(m_in.data_ptr(), rng.data_ptr(),
+                                                                              nrun.data_ptr(), B, H, N, d, sh))
+                rows = B * H * T
+                rec["list_bytes_written"] = int(cnt.sum().item()) * 2 + rows * 4
+                rec["ranges_bytes_written"] = int(nrun.sum().item()) * 4 + rows * 4
+                rec["mean_runs_per_query_tile"] = float(nrun.float().mean().item())
             per_step.append(rec)
             m_in, m_out = m_out, m_in
             tr.advance()

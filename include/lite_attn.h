@@ -112,6 +112,24 @@ int lite_mask_to_list(const uint32_t* mask, int16_t* list, int32_t* counts, int 
                       int d, lite_stream_t stream);
 
 /*
+ * lite_mask_to_ranges -- Skip-Mask to range-encoded Skip-List (skill page, Architecture Overview:
+ * "Bitmask (or Skip-List for high sparsity)"; range pairs as in the README's must_do_list: start
+ * inclusive, end exclusive, strictly descending, because key tiles are visited in reverse order).
+ *
+ * For each (b, h, query tile), every maximal run of live key tiles a..b (a <= b, tile indices)
+ * becomes the pair (b, a - 1); pairs are written from the highest run down.
+ *
+ *  mask    in   device uint32 [B, H, T, W], or NULL = nothing skipped (one run T-1 .. 0).
+ *  ranges  out  device int16 [B, H, T, T+1]: the first 2*nruns[...] entries of each row hold
+ *               start_0, end_0, start_1, end_1, ... with start_0 > end_0 >= start_1 + 1 > ...;
+ *               end may be -1. Later entries are untouched. 2-byte aligned.
+ *  nruns   out  device int32 [B, H, T]: number of runs per query tile (0 when all are skipped).
+ *  B, H, N, d   as in lite_attn_fwd (they fix T and W).
+ */
+int lite_mask_to_ranges(const uint32_t* mask, int16_t* ranges, int32_t* nruns, int B, int H, int N,
+                        int d, lite_stream_t stream);
+
+/*
  * lite_schedule -- work order for the persistent attention kernel (no counterpart on the pages;
  * it orders the query tiles that lite_attn_fwd processes).
  *

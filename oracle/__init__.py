@@ -13,6 +13,7 @@ from .lite_attention import (  # noqa: F401
     range_tiles,
     live_key_tiles,
     mask_to_list,
+    mask_to_ranges,
     schedule_order,
     tile_for_head_dim,
 )

@@ -122,6 +122,38 @@ def mask_to_list(mask, T: int) -> Tuple[np.ndarray, np.ndarray]:
     return lists, counts
 
 
+def mask_to_ranges(mask, T: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Range-encoded Skip-List (skill page, Architecture Overview: "Skip-List for high sparsity";
+    pairs in the README's must_do_list convention: start inclusive, end exclusive, descending).
+
+    Every maximal run of live key tiles a..b of a query tile becomes the pair (b, a - 1), runs from
+    the highest down. Returns (ranges int16 [B,H,T,T+1], nruns int32 [B,H,T]); unused entries are
+    -2 (a value no range entry takes).
+    """
+    m = _as_u32(mask)
+    B, H, T_, _ = m.shape
+    assert T_ == T
+    ranges = np.full((B, H, T, T + 1), -2, dtype=np.int16)
+    nruns = np.zeros((B, H, T), dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            for i in range(T):
+                live = set(live_key_tiles(m, b, h, i, T))
+                pairs = []
+                j = T - 1
+                while j >= 0:
+                    if j in live:
+                        top = j
+                        while j >= 0 and j in live:
+                            j -= 1
+                        pairs += [top, j]  # j is now one below the run (a - 1)
+                    else:
+                        j -= 1
+                nruns[b, h, i] = len(pairs) // 2
+                ranges[b, h, i, : len(pairs)] = pairs
+    return ranges, nruns
+
+
 def schedule_order(counts) -> np.ndarray:
     """Work order over query-tile rows (flattened (b*H + h)*T + i).
 

@@ -390,6 +390,22 @@ int lite_mask_to_list(const uint32_t* mask, int16_t* list, int32_t* counts, int 
   return cudaGetLastError() == cudaSuccess ? LITE_OK : LITE_ERR_CUDA;
 }
 
+int lite_mask_to_ranges(const uint32_t* mask, int16_t* ranges, int32_t* nruns, int B, int H, int N, int d,
+                        lite_stream_t stream) {
+  if (!ranges || !nruns) return LITE_ERR_INVALID_ARG;
+  int st = check_shapes(B, H, N, d);
+  if (st) return st;
+  if (reinterpret_cast<uintptr_t>(ranges) & 1u || reinterpret_cast<uintptr_t>(nruns) & 3u ||
+      reinterpret_cast<uintptr_t>(mask) & 3u)
+    return LITE_ERR_UNSUPPORTED;
+  DeviceCache* dc = nullptr;
+  if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
+  const int t = tile_for(d), T = (N + t - 1) / t, W = (T + 31) / 32;
+  const int rows = B * H * T;
+  lite::lite_ranges_kernel<<<(rows + 7) / 8, 256, 0, as_stream(stream)>>>(mask, ranges, nruns, rows, T, W);
+  return cudaGetLastError() == cudaSuccess ? LITE_OK : LITE_ERR_CUDA;
+}
+
 int lite_schedule(const int32_t* counts, int32_t* order, int B, int H, int T, lite_stream_t stream) {
   if (!counts || !order || B <= 0 || H <= 0 || T <= 0) return LITE_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * H > 8192 || T > kMaxT) return LITE_ERR_UNSUPPORTED;

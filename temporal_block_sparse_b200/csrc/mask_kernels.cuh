@@ -58,6 +58,52 @@ __global__ void __launch_bounds__(256) lite_compact_kernel(const uint32_t* mask_
   if (lane == 0) counts[row] = count;
 }
 
+// Skip-Mask -> range-encoded Skip-List ("Lite Attention Temporal Sparse" skill page, Architecture
+// Overview: "Bitmask (or Skip-List for high sparsity)"; README must_do_list convention for ranges:
+// pairs (start inclusive, end exclusive) in strictly descending order, iterated in reverse).
+// A run of live key tiles a..b (a <= b) becomes the pair (b, a - 1). One warp per (b, h, query
+// tile), words from the top down, lane l owns key tile 32w + 31 - l. A live tile opens a run when
+// the tile above it is not live and closes one when the tile below is not live; ballots of both
+// flags and their prefix popcounts place each lane's start / end entries in order. The tile above
+// lane 0 is the previous word's lane 31 (carried); the tile below lane 31 is bit 31 of the next
+// lower word (read ahead).
+__global__ void __launch_bounds__(256) lite_ranges_kernel(const uint32_t* __restrict__ mask, int16_t* __restrict__ ranges,
+                                                         int32_t* __restrict__ nruns, int rows, int T, int W) {
+  const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp_global >= rows) return;
+  const size_t row = size_t(warp_global);
+  const int R = T + 1;  // entries per row: at most 2 * ceil(T / 2) <= T + 1
+  const uint32_t tail_mask = (T & 31) ? ((1u << (T & 31)) - 1u) : 0xffffffffu;
+  const uint32_t below_me = (1u << lane) - 1u;  // lanes with a higher tile index
+  auto live_bits = [&](int w) -> uint32_t {     // bit i set = tile 32w + i live
+    uint32_t word = mask ? mask[row * W + w] : 0u;
+    uint32_t valid = (w == W - 1) ? tail_mask : 0xffffffffu;
+    return ~word & valid;
+  };
+  int count = 0;
+  bool above_live = false;  // tile 32(w+1) (lane 31 of the word above)
+  uint32_t cur = live_bits(W - 1);
+  for (int w = W - 1; w >= 0; --w) {
+    const uint32_t next = w > 0 ? live_bits(w - 1) : 0u;
+    const int j = w * 32 + 31 - lane;
+    const bool live = (cur >> (31 - lane)) & 1u;
+    const bool up = lane == 0 ? above_live : ((cur >> (32 - lane)) & 1u);      // tile j + 1
+    const bool down = lane == 31 ? ((next >> 31) & 1u) : ((cur >> (30 - lane)) & 1u);  // tile j - 1
+    const bool start = live && !up;
+    const bool end = live && !down;
+    const uint32_t bs = __ballot_sync(0xffffffffu, start);
+    const uint32_t be = __ballot_sync(0xffffffffu, end);
+    const int off = count + __popc(bs & below_me) + __popc(be & below_me);
+    if (start) ranges[row * R + off] = int16_t(j);
+    if (end) ranges[row * R + off + (start ? 1 : 0)] = int16_t(j - 1);
+    count += __popc(bs) + __popc(be);
+    above_live = cur & 1u;
+    cur = next;
+  }
+  if (lane == 0) nruns[row] = count / 2;
+}
+
 // smem: totals[BH] ints, then counts of this head [T] ints
 __global__ void __launch_bounds__(512) lite_schedule_kernel(const int32_t* __restrict__ counts,
                                                            int32_t* __restrict__ order, int BH, int T) {

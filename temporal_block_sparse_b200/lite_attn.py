@@ -49,6 +49,7 @@ SIGNATURES = {
     "lite_attn_dense_ex": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P], _I),
     "lite_lse_merge": ([_P, _P, _I, _P, _P, _I, _I, _I, _I, _P], _I),
     "lite_dropped_mass": ([_P, _P, _P, _P, _I, _I, _I, _P], _I),
+    "lite_mask_to_ranges": ([_P, _P, _P, _I, _I, _I, _I, _P], _I),
 }
 MAX_MERGE_PARTS = 8
 
@@ -324,3 +325,17 @@ def lite_dropped_mass(lse_live: torch.Tensor, lse_full: torch.Tensor, row_mass: 
                                   N, _stream_handle(stream))
     _check("lite_dropped_mass", st)
     return row_mass, stats
+
+
+def lite_mask_to_ranges(mask: Optional[torch.Tensor], B: int, H: int, N: int, d: int, device=None, stream=None):
+    """Range-encoded Skip-List of a mask: (ranges int16 [B, H, T, T+1], nruns int32 [B, H, T]); row r
+    holds nruns[r] (start, end) pairs of live key-tile runs, highest first (end exclusive)."""
+    _, T, _ = lite_mask_geometry(N, d)
+    dev = mask.device if mask is not None else (device or "cuda")
+    if mask is not None:
+        _check_masks(mask)
+    ranges = torch.empty((B, H, T, T + 1), dtype=torch.int16, device=dev)
+    nruns = torch.empty((B, H, T), dtype=torch.int32, device=dev)
+    st = load().lite_mask_to_ranges(_ptr(mask), ranges.data_ptr(), nruns.data_ptr(), B, H, N, d, _stream_handle(stream))
+    _check("lite_mask_to_ranges", st)
+    return ranges, nruns

@@ -27,7 +27,7 @@ def test_header_declares_the_abi():
     names = declared_functions()
     for expected in ("lite_attn_fwd", "lite_attn_dense", "lite_mask_to_list", "lite_mask_geometry",
                      "lite_get_device_status", "lite_status_string", "lite_schedule", "lite_attn_fwd_ex",
-                     "lite_attn_dense_ex", "lite_lse_merge", "lite_dropped_mass"):
+                     "lite_attn_dense_ex", "lite_lse_merge", "lite_dropped_mass", "lite_mask_to_ranges"):
         assert expected in names
 
 
@@ -199,3 +199,14 @@ def test_dropped_mass_argument_checks():
     assert f(FAKE, FAKE, None, FAKE, 1, 1, -3, None) == la.LITE_ERR_INVALID_ARG
     assert f(FAKE + 2, FAKE, None, FAKE, 1, 1, 8, None) == la.LITE_ERR_UNSUPPORTED
     assert f(FAKE, FAKE, FAKE + 1, FAKE, 1, 1, 8, None) == la.LITE_ERR_UNSUPPORTED
+
+
+def test_mask_to_ranges_argument_checks():
+    f = la.load().lite_mask_to_ranges
+    assert f(None, None, FAKE, 1, 1, 256, 128, None) == la.LITE_ERR_INVALID_ARG
+    assert f(None, FAKE, None, 1, 1, 256, 128, None) == la.LITE_ERR_INVALID_ARG
+    assert f(None, FAKE, FAKE, 0, 1, 256, 128, None) == la.LITE_ERR_INVALID_ARG
+    assert f(None, FAKE, FAKE, 1, 1, 256, 96, None) == la.LITE_ERR_UNSUPPORTED
+    assert f(None, FAKE + 1, FAKE, 1, 1, 256, 128, None) == la.LITE_ERR_UNSUPPORTED
+    assert f(FAKE + 2, FAKE, FAKE, 1, 1, 256, 128, None) == la.LITE_ERR_UNSUPPORTED
+    assert f(None, FAKE, FAKE, 1, 1, 4096 * 128 + 1, 128, None) == la.LITE_ERR_UNSUPPORTED
