@@ -127,9 +127,9 @@ struct AttnCfg {
 // Control block in shared memory (barriers are 8-byte mbarrier objects).
 struct alignas(8) AttnCtl {
   uint64_t q_full, q_empty;
-  uint64_t k_full[2], v_full[3];     // K_t (stage t%2) / V_t (stage t%3) landed
+  uint64_t kv_full[2];               // load bundle t landed: K_t (stage t%2) and V_{t-1} (stage (t-1)%3)
   uint64_t s_full[2];                // S_t ready (buffer t%2, one warpgroup each)
-  uint64_t p_lo[2], p_hi[2];         // first / second half of P_t's key columns written
+  uint64_t p_full[2];                // P_t written (buffer t%2)
   uint64_t pv_done[2];               // last PV of group g in an item finished (accumulator g)
   uint64_t mx_full[4], mx_empty[4];  // row maxima of tile t posted in / read from mailbox slot t%4
   uint64_t o_free;                   // epilogue has read both O accumulators
@@ -264,15 +264,13 @@ __global__ void __launch_bounds__(320, 1)
     ptx::mbar_init(BAR(q_full), 1);
     ptx::mbar_init(BAR(q_empty), 1);
     for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(BAR(k_full[b]), 1);
+      ptx::mbar_init(BAR(kv_full[b]), 1);
       ptx::mbar_init(BAR(s_full[b]), 1);
-      ptx::mbar_init(BAR(p_lo[b]), 128);
-      ptx::mbar_init(BAR(p_hi[b]), 128);
+      ptx::mbar_init(BAR(p_full[b]), 128);
       ptx::mbar_init(BAR(pv_done[b]), 1);
       ptx::mbar_init(BAR(item_full[b]), 1);
       ptx::mbar_init(BAR(item_empty[b]), 9);  // MMA thread + one lane of each softmax warp
     }
-    for (int b = 0; b < 3; ++b) ptx::mbar_init(BAR(v_full[b]), 1);
     for (int b = 0; b < 4; ++b) {
       ptx::mbar_init(BAR(mx_full[b]), 128);
       ptx::mbar_init(BAR(mx_empty[b]), 128);
@@ -310,12 +308,34 @@ __global__ void __launch_bounds__(320, 1)
   // away from the awaited one, so the parity waits are exact.
   if (warp == 0) {
     // ------------------------------------------------------------------------- TMA producer
+    // Load bundle t carries K_t (stage t%2, last read by QK_{t-2}) and V_{t-1} (stage (t-1)%3, last
+    // read by PV_{t-4}, which the MMA thread issues before QK_{t-2}); one wait for QK_{t-2} frees
+    // both, and the MMA thread waits once per tile for the bundle. Bundles follow the CTA's tile
+    // sequence across items; one last bundle carries only the final V.
     if (lane == 0) {
       uint32_t t = 0, items = 0, qn = 0;
       bool ok = true;
       // last armed phase of each full barrier, so that every issued load can be drained at exit
-      bool q_armed = false, k_armed[2] = {false, false}, v_armed[3] = {false, false, false};
-      uint32_t q_par = 0, k_par[2] = {0, 0}, v_par[3] = {0, 0, 0};
+      bool q_armed = false, kv_armed[2] = {false, false};
+      uint32_t q_par = 0, kv_par[2] = {0, 0};
+      int pj = 0, ph = 0, pb = 0;  // coordinates of tile t-1
+      // s_full of buffer t%2 next completes with QK_t, which needs this bundle: the wait is exact
+      auto bundle = [&](bool with_k, int j, int h, int b) -> bool {
+        LITE_TRACE(0, 0, t);
+        if (t >= 2 && !wt.wait(BAR(s_full[t & 1]), ((t - 2) >> 1) & 1)) return false;
+        const uint32_t bar = BAR(kv_full[t & 1]);
+        ptx::mbar_arrive_expect_tx(bar, (with_k ? C::KV_TX : 0u) + (t >= 1 ? C::KV_TX : 0u));
+        if (with_k) ptx::tma_load_5d(sK + (t & 1) * C::KV_BYTES, &tmK, bar, 0, j * BN, 0, h, b);
+        if (t >= 1) ptx::tma_load_5d(sV + ((t - 1) % 3) * C::KV_BYTES, &tmV, bar, 0, pj * BN, 0, ph, pb);
+        kv_armed[t & 1] = true;
+        kv_par[t & 1] = (t >> 1) & 1;
+        LITE_TRACE(0, 1, t);
+        pj = j;
+        ph = h;
+        pb = b;
+        ++t;
+        return true;
+      };
       while (ok) {
         const int slot = items & 1;
         if (items >= 2) ok = wt.wait(BAR(item_empty[slot]), ((items >> 1) - 1) & 1);
@@ -329,6 +349,7 @@ __global__ void __launch_bounds__(320, 1)
         if (item < 0) break;
         const ItemInfo it = decode_item(p, item);
         if (it.n == 0) continue;
+        // Q is read by one item's QKs; q_empty is committed after the item's last QK
         if (qn >= 1) ok = wt.wait(BAR(q_empty), (qn - 1) & 1);
         if (!ok) break;
         ptx::mbar_arrive_expect_tx(BAR(q_full), C::Q_TX);
@@ -336,53 +357,59 @@ __global__ void __launch_bounds__(320, 1)
         q_armed = true;
         q_par = qn & 1;
         ++qn;
-        for (int idx = 0; idx < it.n && ok; ++idx, ++t) {
-          const int j = key_entry(p, it.row, idx) & kListIndexMask;
-          // K stage t%2 is free once QK_{t-2} finished. V stage t%3 is free once PV_{t-3} finished,
-          // which is implied by QK_{t-1} finishing: the MMA thread issues PV_{t-3} before QK_{t-1}
-          // and a commit covers every earlier MMA. The s_full barrier of a buffer can only move past
-          // the awaited phase after a K load this thread has not issued yet, so the waits are exact.
-          LITE_TRACE(0, 0, t);
-          if (t >= 2) ok = wt.wait(BAR(s_full[t & 1]), ((t - 2) >> 1) & 1);
-          if (!ok) break;
-          ptx::mbar_arrive_expect_tx(BAR(k_full[t & 1]), C::KV_TX);
-          ptx::tma_load_5d(sK + (t & 1) * C::KV_BYTES, &tmK, BAR(k_full[t & 1]), 0, j * BN, 0, it.h, it.b);
-          LITE_TRACE(0, 1, t);
-          k_armed[t & 1] = true;
-          k_par[t & 1] = (t >> 1) & 1;
-          const uint32_t vs = t % 3;
-          if (t >= 3) ok = wt.wait(BAR(s_full[(t - 1) & 1]), ((t - 1) >> 1) & 1);
-          if (!ok) break;
-          ptx::mbar_arrive_expect_tx(BAR(v_full[vs]), C::KV_TX);
-          ptx::tma_load_5d(sV + vs * C::KV_BYTES, &tmV, BAR(v_full[vs]), 0, j * BN, 0, it.h, it.b);
-          LITE_TRACE(0, 3, t);
-          v_armed[vs] = true;
-          v_par[vs] = (t / 3) & 1;
-        }
+        for (int idx = 0; idx < it.n && ok; ++idx)
+          ok = bundle(true, key_entry(p, it.row, idx) & kListIndexMask, it.h, it.b);
       }
+      if (ok && t >= 1) bundle(false, 0, 0, 0);  // V of the last tile
       // Drain: every issued TMA load has landed before this thread leaves (no other thread arms these
       // barriers, so the last armed phase is the one to wait for).
       if (q_armed) wt.wait_drain(BAR(q_full), q_par);
       for (int b = 0; b < 2; ++b)
-        if (k_armed[b]) wt.wait_drain(BAR(k_full[b]), k_par[b]);
-      for (int b = 0; b < 3; ++b)
-        if (v_armed[b]) wt.wait_drain(BAR(v_full[b]), v_par[b]);
+        if (kv_armed[b]) wt.wait_drain(BAR(kv_full[b]), kv_par[b]);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------------- MMA issuer
-    // The tensor pipe only buffers about 100 cycles of issue gaps, so this loop is kept lean:
-    // descriptors are built once and advanced by 32-bit adds, and per tile there are three waits
-    // (K, P, V) and one commit.
+    // One thread issues, over the CTA's tile sequence (continuously across items):
+    //   QK_t:      S_{t%2} = Q K_t^T          after load bundle t (K_t, V_{t-1}) landed
+    //   PV_{t-1}:  O_{(t-1)%2} += P_{t-1} V_{t-1}   after the softmax released P_{t-1}
+    // Per tile that is two waits, two fences and one commit; the softmax releases P well ahead of
+    // this point, so the waits rarely block. QK_{t+2} reuses S buffer t%2 after PV_t read P_t from
+    // it: MMAs of this thread run in issue order.
     if (lane == 0) {
-      uint32_t t0 = 0, items = 0, qn = 0;
+      uint32_t t = 0, items = 0, qn = 0;
       bool ok = true;
       bool stalled = false;
+      // the tile whose PV is pending: its item number, index in the item and the item's tile count
+      uint32_t pend_item = 0;
+      int pend_idx = 0, pend_n = 0;
       // 128B-swizzled K-major operands advance 32 bytes (>> 4 = 2) per K=16 step inside an atom;
       // V (MN-major) advances 16 rows = 2048 bytes (>> 4 = 128) per step.
       const uint64_t q_desc = umma_desc_sw128(sQ, 16, 1024);
       const uint64_t k_desc0 = umma_desc_sw128(sK, 16, 1024);
       const uint64_t v_desc0 = umma_desc_sw128(sV, C::KV_CHUNK, 1024);
+      auto issue_pv = [&](uint32_t u) -> bool {
+        // the first PV of an item overwrites O_0 / O_1 (the first two, one per accumulator): the
+        // previous item's epilogue must have read both (o_free: one phase per item, exact because
+        // the next phase needs this item's PVs)
+        if (pend_idx == 0 && pend_item >= 1 && !wt.wait(BAR(o_free), (pend_item - 1) & 1)) return false;
+        LITE_TRACE(1, 3, u);
+        // p_full of buffer u%2 next completes for tile u+2, whose S needs QK_{u+2}, issued after this
+        if (!wt.wait(BAR(p_full[u & 1]), (u >> 1) & 1)) return false;
+        LITE_TRACE(1, 4, u);
+        ptx::tc_fence_after();
+        const uint32_t p_tmem = tmem + C::S_COL + (u & 1) * BN;
+        const uint32_t o_tmem = tmem + C::O_COL + (u & 1) * D;
+        const uint64_t vd = v_desc0 + uint64_t(((u % 3) * C::KV_BYTES) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + uint64_t(kk * 128), C::IDESC_PV,
+                      (pend_idx < 2 && kk == 0) ? 0u : 1u);
+        // the epilogue of group u%2 waits for the item's last PV into its accumulator
+        if (pend_idx >= pend_n - 2) ptx::mma_commit(BAR(pv_done[u & 1]));
+        LITE_TRACE(1, 6, u);
+        return true;
+      };
       while (ok) {
         const int slot = items & 1;
         ok = wt.wait(BAR(item_full[slot]), (items >> 1) & 1);
@@ -403,63 +430,41 @@ __global__ void __launch_bounds__(320, 1)
           ok = false;
           break;
         }
+        // q_full completes once per item; the next load waits for this item's q_empty commit
         ok = wt.wait(BAR(q_full), qn & 1);
         if (!ok) break;
         ptx::tc_fence_after();
-        // tiles idx = 0 .. n: QK_idx (idx < n), then PV_{idx-1} (idx >= 1)
-        for (int idx = 0; idx <= it.n && ok; ++idx) {
-          if (idx < it.n) {
-            const uint32_t t = t0 + idx;
-            LITE_TRACE(1, 0, t);
-            if (!wt.wait(BAR(k_full[t & 1]), (t >> 1) & 1)) { ok = false; break; }
-            LITE_TRACE(1, 1, t);
-            ptx::tc_fence_after();
-            const uint64_t kd = k_desc0 + uint64_t(((t & 1) * C::KV_BYTES) >> 4);
-            const uint32_t s_tmem = tmem + C::S_COL + (t & 1) * BN;
+        for (int idx = 0; idx < it.n && ok; ++idx, ++t) {
+          // kv_full of this slot next completes for bundle t+2, loaded after QK_t finished
+          LITE_TRACE(1, 0, t);
+          if (!wt.wait(BAR(kv_full[t & 1]), (t >> 1) & 1)) { ok = false; break; }
+          LITE_TRACE(1, 1, t);
+          ptx::tc_fence_after();
+          const uint64_t kd = k_desc0 + uint64_t(((t & 1) * C::KV_BYTES) >> 4);
+          const uint32_t s_tmem = tmem + C::S_COL + (t & 1) * BN;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint64_t off = uint64_t((kk >> 2) * (C::Q_CHUNK >> 4) + (kk & 3) * 2);
-              const uint64_t offk = uint64_t((kk >> 2) * (C::KV_CHUNK >> 4) + (kk & 3) * 2);
-              ptx::mma_ss(s_tmem, q_desc + off, kd + offk, C::IDESC_QK, kk > 0 ? 1u : 0u);
-            }
-            ptx::mma_commit(BAR(s_full[t & 1]));
-            LITE_TRACE(1, 2, t);
-            if (idx == it.n - 1) ptx::mma_commit(BAR(q_empty));
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = uint64_t((kk >> 2) * (C::Q_CHUNK >> 4) + (kk & 3) * 2);
+            const uint64_t offk = uint64_t((kk >> 2) * (C::KV_CHUNK >> 4) + (kk & 3) * 2);
+            ptx::mma_ss(s_tmem, q_desc + off, kd + offk, C::IDESC_QK, kk > 0 ? 1u : 0u);
           }
-          if (idx >= 1) {
-            // O_{t%2} += P_t V_t for the previous tile; QK_{t+2} (next iteration but one) reuses
-            // S buffer t%2, and MMAs of this thread run in issue order
-            const int pv = idx - 1;
-            const uint32_t t = t0 + pv;
-            if (pv == 0 && qn >= 1 && !wt.wait(BAR(o_free), (qn - 1) & 1)) { ok = false; break; }
-            LITE_TRACE(1, 3, t);
-            if (!wt.wait(BAR(p_lo[t & 1]), (t >> 1) & 1)) { ok = false; break; }
-            LITE_TRACE(1, 4, t);
-            if (!wt.wait(BAR(v_full[t % 3]), (t / 3) & 1)) { ok = false; break; }
-            LITE_TRACE(1, 5, t);
-            ptx::tc_fence_after();
-            const uint32_t p_tmem = tmem + C::S_COL + (t & 1) * BN;
-            const uint32_t o_tmem = tmem + C::O_COL + (t & 1) * D;
-            const uint64_t vd = v_desc0 + uint64_t(((t % 3) * C::KV_BYTES) >> 4);
-            // the first half of the key columns starts as soon as its P is written; the softmax
-            // computes the second half meanwhile
-#pragma unroll
-            for (int kk = 0; kk < BN / 32; ++kk)
-              ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + uint64_t(kk * 128), C::IDESC_PV,
-                          (pv < 2 && kk == 0) ? 0u : 1u);
-            if (!wt.wait(BAR(p_hi[t & 1]), (t >> 1) & 1)) { ok = false; break; }
-            LITE_TRACE(1, 7, t);
-            ptx::tc_fence_after();
-#pragma unroll
-            for (int kk = BN / 32; kk < BN / 16; ++kk)
-              ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + uint64_t(kk * 128), C::IDESC_PV, 1u);
-            // the epilogue of group t%2 waits for the last PV into its accumulator
-            if (pv >= it.n - 2) ptx::mma_commit(BAR(pv_done[t & 1]));
-            LITE_TRACE(1, 6, t);
-          }
+          ptx::mma_commit(BAR(s_full[t & 1]));
+          if (idx == it.n - 1) ptx::mma_commit(BAR(q_empty));
+          LITE_TRACE(1, 2, t);
+          if (t >= 1 && !issue_pv(t - 1)) { ok = false; break; }
+          pend_item = qn;
+          pend_idx = idx;
+          pend_n = it.n;
         }
-        t0 += it.n;
         ++qn;
+      }
+      // the last tile's PV, once the final bundle (its V) has landed
+      if (ok && t >= 1) {
+        ok = wt.wait(BAR(kv_full[t & 1]), (t >> 1) & 1);
+        if (ok) {
+          ptx::tc_fence_after();
+          issue_pv(t - 1);
+        }
       }
       // all issued tensor-core work must finish before TMEM is released
       ptx::mma_commit(BAR(drain));
@@ -537,11 +542,6 @@ __global__ void __launch_bounds__(320, 1)
         }
         const float loc = ptx::fmax3(m0, m1, fmaxf(m2, m3)) * p.scale_log2;
         if (r == 0) LITE_TRACE(2 + grp, 2, t);
-        // post this tile's row maxima for the group that takes tile t+1 (they enter its QK-Skip
-        // running max). Slot t%4 is refilled every four tiles, after its reader took tile t-4's.
-        if (t >= 4) wt.wait(BAR(mx_empty[t & 3]), ((t >> 2) - 1) & 1);
-        mailbox[(t & 3) * 128 + r] = loc;
-        ptx::mbar_arrive(BAR(mx_full[t & 3]));
         // lazy rescale of this group's accumulator: move the reference only when the tile max
         // exceeds it by more than 8 (log2 units). The previous PV into this accumulator (tile t-2)
         // was issued before QK_t, so it has completed now that S_t is ready; the rescaled O is
@@ -566,34 +566,36 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
         // P = 2^(s*scale*log2e - m_used) as bf16 pairs over the S columns (chunk c of 32 key
-        // columns -> TMEM columns [16c, 16c+16)), released in two halves of the key columns so
-        // that the first half of PV runs while the second half is exponentiated. Packed fp32x2
-        // arithmetic for the affine step and the row sum; one column pair in four is exponentiated
-        // on the FMA pipe, the rest on MUFU.
+        // columns -> TMEM columns [16c, 16c+16)), released to the MMA thread in one piece. Packed
+        // fp32x2 arithmetic for the affine step and the row sum; one column pair in four is
+        // exponentiated on the FMA pipe, the rest on MUFU.
         const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
         const float2 nm2 = make_float2(-m_used, -m_used);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int x = 0; x < 16; ++x) {
-              const float2 a = __ffma2_rn(make_float2(s[32 * c + 2 * x], s[32 * c + 2 * x + 1]), sc2, nm2);
-              const float2 pp = ((x & 3) == 3) ? exp2_poly2(a) : make_float2(ptx::ex2(a.x), ptx::ex2(a.y));
-              acc[x & 3] = __fadd2_rn(acc[x & 3], pp);
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(pp.x, pp.y);
-              pk[x] = *reinterpret_cast<uint32_t*>(&h2);
-            }
-            ptx::tmem_st16(s_tmem + c * 16, pk);
+          for (int x = 0; x < 16; ++x) {
+            const float2 a = __ffma2_rn(make_float2(s[32 * c + 2 * x], s[32 * c + 2 * x + 1]), sc2, nm2);
+            const float2 pp = ((x & 3) == 3) ? exp2_poly2(a) : make_float2(ptx::ex2(a.x), ptx::ex2(a.y));
+            acc[x & 3] = __fadd2_rn(acc[x & 3], pp);
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(pp.x, pp.y);
+            pk[x] = *reinterpret_cast<uint32_t*>(&h2);
           }
-          ptx::tmem_wait_st();
-          ptx::tc_fence_before();
-          ptx::mbar_arrive(half == 0 ? BAR(p_lo[grp]) : BAR(p_hi[grp]));
-          if (half == 0 && r == 0) LITE_TRACE(2 + grp, 5, t);
+          ptx::tmem_st16(s_tmem + c * 16, pk);
         }
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(BAR(p_full[grp]));
         if (r == 0) LITE_TRACE(2 + grp, 6, t);
+        // Post this tile's row maxima for the group that takes tile t+1; they enter its QK-Skip
+        // running max, which its vote reads after its own P release, so the post is off the path
+        // from S to P here too. Slot t%4 is refilled every four tiles, after its reader took tile t-4's.
+        if (t >= 4) wt.wait(BAR(mx_empty[t & 3]), ((t >> 2) - 1) & 1);
+        mailbox[(t & 3) * 128 + r] = loc;
+        ptx::mbar_arrive(BAR(mx_full[t & 3]));
+        if (r == 0) LITE_TRACE(2 + grp, 7, t);
         const float2 acc2 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
         l += acc2.x + acc2.y;
         // QK-Skip vote, off the path from S to P. The running max over the tiles visited before t
