@@ -700,6 +700,38 @@ def run_calibration_study(args):
     print(json.dumps(line), flush=True)
 
 
+def _load_balance(la, q, k, v, mask, tau):
+    """Per-CTA busy time of the attention kernel on one mask, with the longest-first schedule and with
+    query tiles in their natural order: {order: {kernel_ms, busy max/mean, tiles max/mean}}."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    buf = torch.zeros((sms, 3), dtype=torch.int64, device="cuda")
+    m_out = torch.empty_like(mask)
+    out = {}
+    for name, sched in (("longest_first", 1), ("natural", 0)):
+        la.lite_set_option(la.LITE_OPT_SCHEDULE, sched)
+        step = lambda: la.lite_attn_fwd(q, k, v, mask, m_out, tau=tau)
+        step()
+        ms = min(_time_call(step), _time_call(step))
+        buf.zero_()
+        la.lite_set_cta_timing(buf)
+        step()
+        torch.cuda.synchronize()
+        la.lite_set_cta_timing(None)
+        rec = buf.cpu().double()
+        used = rec[:, 1] > 0
+        busy = (rec[used, 1] - rec[used, 0]) * 1e-6
+        tiles = rec[used, 2]
+        ends = rec[used, 1] * 1e-6
+        # every CTA takes work until none is left, so start-to-end times match by construction; the
+        # spread of end times (how early the first CTA ran dry) and of tiles per CTA show the balance
+        out[name] = {"kernel_ms": ms, "ctas": int(used.sum()), "busy_ms_mean": float(busy.mean()),
+                     "end_spread_ms": float(ends.max() - ends.min()),
+                     "tiles_max_over_mean": float(tiles.max() / tiles.mean()),
+                     "tiles_min_over_mean": float(tiles.min() / tiles.mean())}
+    la.lite_set_option(la.LITE_OPT_SCHEDULE, 1)
+    return out
+
+
 def run_study(args):
     """Threshold sweep and stress reports (one JSON line per run; not the headline metric)."""
     from temporal_block_sparse_b200 import lite_attn as la
@@ -773,6 +805,9 @@ def run_study(args):
             per_step.append(rec)
             m_in, m_out = m_out, m_in
             tr.advance()
+        balance = None
+        if args.study == "stress":
+            balance = _load_balance(la, q, k, v, m_in, tau)
         assert la.lite_get_device_status() == 0
         # linearity: step time against live fraction (least squares), over steps with any skipping
         xs = [1 - r["skipped"] for r in per_step]
@@ -790,6 +825,8 @@ def run_study(args):
         line = {"study": args.study, "workload": f"{base.name}: B={B} H={H} N={N} d={d}", "tau": tau,
                 "steps": steps, "dense_ms": dense_ms, "final_skipped": per_step[-1]["skipped"],
                 "time_vs_live_fraction_fit": fit, "skipped_mass_bound_step0": bound, "per_step": per_step}
+        if balance is not None:
+            line["load_balance_final_mask"] = balance
         print(json.dumps(line), flush=True)
         del tr
 

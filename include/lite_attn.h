@@ -167,10 +167,22 @@ const char* lite_status_string(int status);
  *  LITE_OPT_DEBUG_STALL    1 = test hook: the MMA warp of every CTA withholds its first tile, so
  *                          the waits that depend on it run out their limit (no fault, no hang).
  *  LITE_OPT_MAX_CTAS       cap on the persistent grid size (0 = one CTA per SM).
+ *  LITE_OPT_SCHEDULE       1 (default) = lite_attn_fwd* hand out query tiles in the longest-first
+ *                          order of lite_schedule; 0 = in their natural (b, h, tile) order, for
+ *                          measuring what the schedule buys. Results are identical either way.
  * Returns LITE_ERR_INVALID_ARG for an unknown option or out-of-range value.
  */
-enum { LITE_OPT_WAIT_LIMIT_NS = 1, LITE_OPT_DEBUG_STALL = 2, LITE_OPT_MAX_CTAS = 3 };
+enum { LITE_OPT_WAIT_LIMIT_NS = 1, LITE_OPT_DEBUG_STALL = 2, LITE_OPT_MAX_CTAS = 3, LITE_OPT_SCHEDULE = 4 };
 int lite_set_option(int option, long long value);
+
+/*
+ * lite_set_cta_timing -- measurement hook for load balance. While set, every attention kernel
+ * launch writes, for each CTA b < capacity, buf[3b] = its start time, buf[3b+1] = its end time
+ * (both the GPU's global nanosecond timer) and buf[3b+2] = the number of live tiles it processed.
+ * buf is caller-owned device memory of 3 * capacity uint64 values (8-byte aligned), or NULL with
+ * capacity 0 to stop. Host state, like lite_set_kernel_events.
+ */
+int lite_set_cta_timing(void* buf, int capacity);
 
 /*
  * lite_set_kernel_events -- measurement hook. While set, every lite_attn_fwd* / lite_attn_dense*

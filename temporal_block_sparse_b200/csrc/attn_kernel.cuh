@@ -64,6 +64,8 @@ struct AttnParams {
   int skip_test;            // 1: run the QK-Skip vote and record flags
   unsigned long long wait_limit_ns;
   int debug_stall;          // test hook: MMA warp withholds its first tile
+  unsigned long long* cta_times;  // measurement hook: [cta_cap][3] {start ns, end ns, tiles}, or null
+  int cta_cap;
 #ifdef LITE_ATTN_TRACE
   long long* trace;         // [4 CTAs][4 roles][8 events][512 tiles] clock64 stamps
 #endif
@@ -138,6 +140,7 @@ struct alignas(8) AttnCtl {
   uint32_t tmem_base;
   int item[2];
   int abort;
+  uint32_t tiles;                    // live tiles this CTA processed (measurement hook)
 };
 
 // UMMA shared-memory descriptor, 128-byte swizzle (layout type 2, bits 61-63), version 1 (bit 46).
@@ -260,6 +263,7 @@ __global__ void __launch_bounds__(320, 1)
 
 #define BAR(x) ptx::smem_addr(&ctl->x)
 
+  const uint64_t t_start = ptx::globaltimer();
   if (threadIdx.x == 0) {
     ptx::mbar_init(BAR(q_full), 1);
     ptx::mbar_init(BAR(q_empty), 1);
@@ -360,6 +364,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int idx = 0; idx < it.n && ok; ++idx)
           ok = bundle(true, key_entry(p, it.row, idx) & kListIndexMask, it.h, it.b);
       }
+      ctl->tiles = t;
       if (ok && t >= 1) bundle(false, 0, 0, 0);  // V of the last tile
       // Drain: every issued TMA load has landed before this thread leaves (no other thread arms these
       // barriers, so the last armed phase is the one to wait for).
@@ -678,6 +683,12 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && p.cta_times && int(blockIdx.x) < p.cta_cap) {
+    unsigned long long* rec = p.cta_times + 3 * size_t(blockIdx.x);
+    rec[0] = t_start;
+    rec[1] = ptx::globaltimer();
+    rec[2] = ctl->tiles;
   }
 }
 

@@ -31,8 +31,11 @@ struct Options {
   unsigned long long wait_limit_ns = 4000000000ull;
   int debug_stall = 0;
   int max_ctas = 0;
+  int schedule = 1;
 };
 Options g_opt;
+unsigned long long* g_cta_times = nullptr;
+int g_cta_cap = 0;
 cudaEvent_t g_ev_before = nullptr;
 cudaEvent_t g_ev_after = nullptr;
 #ifdef LITE_ATTN_TRACE
@@ -187,6 +190,8 @@ lite::AttnParams base_params(void* o, float* lse, int B, int H, int Nq, int Nk, 
   p.status = dc->status;
   p.wait_limit_ns = g_opt.wait_limit_ns;
   p.debug_stall = g_opt.debug_stall;
+  p.cta_times = g_cta_times;
+  p.cta_cap = g_cta_cap;
 #ifdef LITE_ATTN_TRACE
   p.trace = g_trace;
 #endif
@@ -284,13 +289,15 @@ int enqueue_fwd(DeviceCache* dc, const FwdArgs& a, const lite::RangeBits* ranges
     lite::lite_compact_kernel<false><<<cblocks, 256, 0, s>>>(a.mask_in, a.mask_out, list, counts, rows, Tk, W,
                                                              lite::RangeBits{});
   if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
-  const size_t sm = size_t(a.B * a.H + Tq) * sizeof(int32_t);
-  lite::lite_schedule_kernel<<<a.B * a.H, 512, sm, s>>>(counts, order, a.B * a.H, Tq);
-  if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
+  if (g_opt.schedule) {
+    const size_t sm = size_t(a.B * a.H + Tq) * sizeof(int32_t);
+    lite::lite_schedule_kernel<<<a.B * a.H, 512, sm, s>>>(counts, order, a.B * a.H, Tq);
+    if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
+  }
   p.mask_out = a.mask_out;
   p.list = list;
   p.counts = counts;
-  p.order = order;
+  p.order = g_opt.schedule ? order : nullptr;  // null: rows in their natural order
   p.work_counter = counter;
   p.tau_log2 = a.tau * 1.4426950408889634f;
   p.skip_test = (a.mask_out != nullptr && a.tau > -INFINITY) ? 1 : 0;
@@ -347,6 +354,10 @@ int lite_set_option(int option, long long value) {
       if (value != 0 && value != 1) return LITE_ERR_INVALID_ARG;
       g_opt.debug_stall = static_cast<int>(value);
       return LITE_OK;
+    case LITE_OPT_SCHEDULE:
+      if (value != 0 && value != 1) return LITE_ERR_INVALID_ARG;
+      g_opt.schedule = int(value);
+      return LITE_OK;
     case LITE_OPT_MAX_CTAS:
       if (value < 0 || value > 1000000) return LITE_ERR_INVALID_ARG;
       g_opt.max_ctas = static_cast<int>(value);
@@ -354,6 +365,14 @@ int lite_set_option(int option, long long value) {
     default:
       return LITE_ERR_INVALID_ARG;
   }
+}
+
+int lite_set_cta_timing(void* buf, int capacity) {
+  if ((buf == nullptr) != (capacity == 0) || capacity < 0) return LITE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(buf) & 7u) return LITE_ERR_UNSUPPORTED;
+  g_cta_times = static_cast<unsigned long long*>(buf);
+  g_cta_cap = capacity;
+  return LITE_OK;
 }
 
 int lite_set_kernel_events(void* before, void* after) {

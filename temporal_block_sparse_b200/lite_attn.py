@@ -50,6 +50,7 @@ SIGNATURES = {
     "lite_lse_merge": ([_P, _P, _I, _P, _P, _I, _I, _I, _I, _P], _I),
     "lite_dropped_mass": ([_P, _P, _P, _P, _I, _I, _I, _P], _I),
     "lite_mask_to_ranges": ([_P, _P, _P, _I, _I, _I, _I, _P], _I),
+    "lite_set_cta_timing": ([_P, _I], _I),
 }
 MAX_MERGE_PARTS = 8
 
@@ -339,3 +340,17 @@ def lite_mask_to_ranges(mask: Optional[torch.Tensor], B: int, H: int, N: int, d:
     st = load().lite_mask_to_ranges(_ptr(mask), ranges.data_ptr(), nruns.data_ptr(), B, H, N, d, _stream_handle(stream))
     _check("lite_mask_to_ranges", st)
     return ranges, nruns
+
+
+LITE_OPT_SCHEDULE = 4
+
+
+def lite_set_cta_timing(buf: Optional[torch.Tensor]):
+    """Per-CTA {start ns, end ns, tiles} records of every following attention launch go to buf
+    (int64 [capacity, 3] on the GPU); None stops recording."""
+    if buf is None:
+        _check("lite_set_cta_timing", load().lite_set_cta_timing(None, 0))
+        return
+    if buf.dtype != torch.int64 or buf.dim() != 2 or buf.shape[1] != 3 or not buf.is_contiguous():
+        raise ValueError("buf must be a contiguous int64 [capacity, 3] tensor")
+    _check("lite_set_cta_timing", load().lite_set_cta_timing(buf.data_ptr(), buf.shape[0]))

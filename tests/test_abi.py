@@ -210,3 +210,15 @@ def test_mask_to_ranges_argument_checks():
     assert f(None, FAKE + 1, FAKE, 1, 1, 256, 128, None) == la.LITE_ERR_UNSUPPORTED
     assert f(FAKE + 2, FAKE, FAKE, 1, 1, 256, 128, None) == la.LITE_ERR_UNSUPPORTED
     assert f(None, FAKE, FAKE, 1, 1, 4096 * 128 + 1, 128, None) == la.LITE_ERR_UNSUPPORTED
+
+
+def test_cta_timing_and_schedule_option_checks():
+    lib = la.load()
+    assert lib.lite_set_cta_timing(None, 0) == la.LITE_OK
+    assert lib.lite_set_cta_timing(None, 4) == la.LITE_ERR_INVALID_ARG
+    assert lib.lite_set_cta_timing(FAKE, 0) == la.LITE_ERR_INVALID_ARG
+    assert lib.lite_set_cta_timing(FAKE, -1) == la.LITE_ERR_INVALID_ARG
+    assert lib.lite_set_cta_timing(FAKE + 4, 8) == la.LITE_ERR_UNSUPPORTED
+    assert lib.lite_set_option(la.LITE_OPT_SCHEDULE, 2) == la.LITE_ERR_INVALID_ARG
+    assert lib.lite_set_option(la.LITE_OPT_SCHEDULE, 0) == la.LITE_OK
+    assert lib.lite_set_option(la.LITE_OPT_SCHEDULE, 1) == la.LITE_OK

@@ -1,0 +1,68 @@
+"""The longest-first work order changes only which CTA processes which query tile (needs a B200).
+
+Results (o, lse, mask) are bit-identical with the schedule on and off; the per-CTA timing hook
+accounts for every live tile exactly once.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from temporal_block_sparse_b200 import lite_attn as la
+from temporal_block_sparse_b200 import workload as wl
+
+pytestmark = [pytest.mark.gpu, pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+
+@pytest.fixture(autouse=True)
+def _clean_state():
+    la.load()
+    yield
+    la.lite_set_option(la.LITE_OPT_SCHEDULE, 1)
+    la.lite_set_cta_timing(None)
+    assert la.lite_get_device_status() == 0
+
+
+def _masked_step(seed):
+    w = wl.small_workload(2, 3, 8, 16, 16, 128, steps=2, locality=5.0, tau=-2.0, seed_offset=seed)  # N = 2048
+    tr = wl.Trajectory(w, device="cuda")
+    q, k, v = tr.current()
+    B, N, H, d = q.shape
+    m0 = la.new_mask(B, H, N, d)
+    m1 = torch.empty_like(m0)
+    la.lite_attn_fwd(q, k, v, m0, m1, tau=-2.0)  # a non-uniform mask for the next step
+    tr.advance()
+    return tr.current(), m1
+
+
+def test_schedule_off_gives_identical_results():
+    (q, k, v), m_in = _masked_step(61)
+    outs = []
+    for sched in (1, 0):
+        la.lite_set_option(la.LITE_OPT_SCHEDULE, sched)
+        m_out = torch.empty_like(m_in)
+        o, lse = la.lite_attn_fwd(q, k, v, m_in, m_out, tau=-2.0)
+        torch.cuda.synchronize()
+        outs.append((o.clone(), lse.clone(), m_out.clone()))
+    assert torch.equal(outs[0][0], outs[1][0])
+    assert torch.equal(outs[0][1], outs[1][1])
+    assert torch.equal(outs[0][2], outs[1][2])
+
+
+def test_cta_timing_counts_every_live_tile():
+    (q, k, v), m_in = _masked_step(62)
+    B, N, H, d = q.shape
+    _, T, _ = la.lite_mask_geometry(N, d)
+    _, counts = la.lite_mask_to_list(m_in, B, H, N, d)
+    live = int(counts.sum().item())
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    buf = torch.zeros((sms, 3), dtype=torch.int64, device="cuda")
+    la.lite_set_cta_timing(buf)
+    la.lite_attn_fwd(q, k, v, m_in, torch.empty_like(m_in), tau=-2.0)
+    torch.cuda.synchronize()
+    la.lite_set_cta_timing(None)
+    rec = buf.cpu().numpy()
+    used = rec[:, 1] > 0
+    assert used.sum() == min(sms, B * H * T)
+    assert (rec[used, 1] >= rec[used, 0]).all()
+    assert int(rec[used, 2].sum()) == live
