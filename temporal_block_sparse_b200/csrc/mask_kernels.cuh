@@ -25,7 +25,31 @@ struct RangeBits {
   uint32_t skip[128];  // must-skip (must-do already removed): always skipped
 };
 
-// mask_in may alias mask_out (in-place update): each warp reads a word before it writes it back.
+// Words of one mask row into registers: lane l gets words l, l + 32, l + 64, l + 96 (0 past W;
+// bits >= T of the last word cleared). Rows have at most 128 words (T <= 4096).
+__device__ __forceinline__ void load_row_words(const uint32_t* mask, size_t row, int W, int T, int lane,
+                                               uint32_t (&wr)[4]) {
+  const uint32_t tail_mask = (T & 31) ? ((1u << (T & 31)) - 1u) : 0xffffffffu;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int w = lane + 32 * i;
+    uint32_t v = 0u;
+    if (w < W) {
+      v = mask ? mask[row * W + w] : 0u;
+      if (w == W - 1) v &= tail_mask;
+    }
+    wr[i] = v;
+  }
+}
+
+// Word w of the row, broadcast to the whole warp (w is warp-uniform).
+__device__ __forceinline__ uint32_t row_word(const uint32_t (&wr)[4], int w) {
+  const int i = w >> 5;
+  const uint32_t mine = i == 0 ? wr[0] : (i == 1 ? wr[1] : (i == 2 ? wr[2] : wr[3]));
+  return __shfl_sync(0xffffffffu, mine, w & 31);
+}
+
+// mask_in may alias mask_out (in-place update): each warp reads its row before it writes it back.
 // kRanges: apply RangeBits (live wins over skip and over the mask; tagged entries are never flagged).
 template <bool kRanges>
 __global__ void __launch_bounds__(256) lite_compact_kernel(const uint32_t* mask_in, uint32_t* mask_out,
@@ -35,12 +59,19 @@ __global__ void __launch_bounds__(256) lite_compact_kernel(const uint32_t* mask_
   const int lane = threadIdx.x & 31;
   if (warp_global >= rows) return;
   const size_t row = size_t(warp_global);
-  const uint32_t tail_mask = (T & 31) ? ((1u << (T & 31)) - 1u) : 0xffffffffu;
+  // The row's words are read in one round (lane l holds words l, l+32, l+64, l+96; W <= 128), so
+  // the warp waits for memory once, not once per word; the copy to mask_out is written the same
+  // way. In place (mask_out == mask_in) is safe: every word of the row is read before any write.
+  uint32_t wr[4];
+  load_row_words(mask_in, row, W, T, lane, wr);
+  if (mask_out) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (lane + 32 * i < W) mask_out[row * W + lane + 32 * i] = wr[i];
+  }
   int count = 0;
   for (int w = W - 1; w >= 0; --w) {
-    uint32_t word = mask_in ? mask_in[row * W + w] : 0u;
-    if (w == W - 1) word &= tail_mask;  // bits >= T carry no tile
-    if (mask_out && lane == 0) mask_out[row * W + w] = word;
+    uint32_t word = row_word(wr, w);
     uint32_t forced = 0u;
     if constexpr (kRanges) {
       forced = ranges.live[w];
@@ -76,10 +107,11 @@ __global__ void __launch_bounds__(256) lite_ranges_kernel(const uint32_t* __rest
   const int R = T + 1;  // entries per row: at most 2 * ceil(T / 2) <= T + 1
   const uint32_t tail_mask = (T & 31) ? ((1u << (T & 31)) - 1u) : 0xffffffffu;
   const uint32_t below_me = (1u << lane) - 1u;  // lanes with a higher tile index
+  uint32_t wr[4];
+  load_row_words(mask, row, W, T, lane, wr);   // one round of loads for the whole row
   auto live_bits = [&](int w) -> uint32_t {     // bit i set = tile 32w + i live
-    uint32_t word = mask ? mask[row * W + w] : 0u;
-    uint32_t valid = (w == W - 1) ? tail_mask : 0xffffffffu;
-    return ~word & valid;
+    const uint32_t valid = (w == W - 1) ? tail_mask : 0xffffffffu;
+    return ~row_word(wr, w) & valid;
   };
   int count = 0;
   bool above_live = false;  // tile 32(w+1) (lane 31 of the word above)
