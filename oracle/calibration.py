@@ -13,7 +13,7 @@ Sources (the LiteAttention pages):
   * README, "QK-Skip Algorithm": once marked, a tile is skipped at every later step (the mask only
     grows), so the error a step's flags introduce is carried by every later step.
 
-Readings where the pages are silent (stated again in the design doc):
+Readings where the pages are silent:
   * The multiplier scales the QK-Skip element bound exp(tau): a tile flagged with threshold tau has
     every element below exp(tau) under that step's softmax, so a budget multiplier b corresponds to
     tau + ln(b) (tau_for_budget).
