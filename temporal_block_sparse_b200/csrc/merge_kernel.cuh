@@ -8,12 +8,14 @@
 // A part with lse_p = -inf (no key for that row) has w_p = 0; if every part is -inf the row is 0
 // with lse -inf.
 //
-// HBM-bound: per row it reads P * (2 d + 4) bytes and writes 2 d + 4. Each thread owns 16 bytes
-// (8 bf16) of one row. Rows are walked in memory order of o, (b, n, h), so a warp reads and writes
-// one contiguous 512-byte stretch of every part (d = 128: two rows); the lse values it needs are
-// strided by N but few (24 MB for a 720p layer's two parts), and the n-neighbours that share their
-// sectors are processed right after, out of L2. All parts' loads of a thread are issued before any
-// arithmetic. Index arithmetic is 32-bit (the host refuses B*H*N*d/8 >= 2^31).
+// HBM-bound: per row it reads P * (2 d + 4) bytes and writes 2 d + 4. A thread owns 16-byte pieces
+// (8 bf16) of rows: with two parts, two pieces a grid stride apart per iteration, whose loads are
+// all issued before any arithmetic (64 bytes in flight per thread; more pieces cost more than they
+// gain). Rows are walked in memory order of o, (b, n, h), so a warp reads and writes one contiguous
+// 512-byte stretch of every part (d = 128: two rows); the lse values it needs are strided by N but
+// few (24 MB for a 720p layer's two parts), and the n-neighbours that share their sectors are
+// processed right after, out of L2. Index arithmetic is 32-bit (the host refuses
+// B*H*N*d/8 >= 2^31).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -34,78 +36,95 @@ struct MergeParts {
 // MP >= parts.n bounds the unrolled part loop (2, 4 or 8), so that few parts need few registers
 // and more threads per SM keep more bytes in flight.
 template <int D, int MP>
+__device__ __forceinline__ void merge_one(const MergeParts& parts, const float (&l)[MP], const uint4 (&v)[MP],
+                                          __nv_bfloat16* o, float* lse, size_t off, size_t lrow, bool write_lse) {
+  float m = -INFINITY;
+#pragma unroll
+  for (int p = 0; p < MP; ++p) m = fmaxf(m, l[p]);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float out_lse = -INFINITY;
+  if (m > -INFINITY) {
+    float w[MP];
+    float tot = 0.f;
+#pragma unroll
+    for (int p = 0; p < MP; ++p) {
+      w[p] = (l[p] > -INFINITY) ? expf(l[p] - m) : 0.f;
+      tot += w[p];
+    }
+    const float inv = 1.f / tot;
+#pragma unroll
+    for (int p = 0; p < MP; ++p) {
+      if (w[p] == 0.f) continue;
+      const float wp = w[p] * inv;
+      const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&v[p]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(x[e]);
+        acc[2 * e] = fmaf(wp, f.x, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(wp, f.y, acc[2 * e + 1]);
+      }
+    }
+    out_lse = m + logf(tot);
+  }
+  uint4 res;
+  uint32_t* r = reinterpret_cast<uint32_t*>(&res);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
+    r[e] = *reinterpret_cast<uint32_t*>(&h2);
+  }
+  *reinterpret_cast<uint4*>(o + off) = res;
+  if (lse && write_lse) lse[lrow] = out_lse;
+}
+
+// o / lse may alias a part's buffers (in-place merge): every thread reads all of its inputs, the
+// warp (which holds whole rows) synchronises, then each thread writes only elements it has read.
+// MP >= parts.n bounds the unrolled part loop (2, 4 or 8), so that few parts need few registers.
+// Each thread takes U 16-byte pieces a grid stride apart per iteration and issues all their loads
+// before any arithmetic, so U * parts * 16 bytes are in flight per thread.
+template <int D, int MP>
 __global__ void __launch_bounds__(256) lite_lse_merge_kernel(const MergeParts parts, __nv_bfloat16* o, float* lse,
                                                              int B, int H, int N) {
   constexpr int G = D / 8;  // threads per row
+  constexpr int U = MP <= 2 ? 2 : 1;
   const uint32_t total = uint32_t(B) * H * N * G;
   const uint32_t stride = gridDim.x * blockDim.x;
   // the loop bound is uniform over a warp (whole warps step together), so __syncwarp is legal
   const uint32_t warp_base0 = (blockIdx.x * blockDim.x + threadIdx.x) & ~31u;
   const uint32_t lane = threadIdx.x & 31;
-  for (uint32_t base = warp_base0; base < total; base += stride) {
-    const uint32_t gid = base + lane;
-    const bool valid = gid < total;
-    const uint32_t row = valid ? gid / G : 0;  // (b * N + n) * H + h: the memory order of o
-    const uint32_t g = gid - row * G;
-    const uint32_t bn = row / uint32_t(H);
-    const uint32_t h = row - bn * uint32_t(H);
-    const uint32_t b = bn / uint32_t(N);
-    const uint32_t n = bn - b * uint32_t(N);
-    const size_t off = size_t(row) * D + g * 8;
-    const size_t lrow = (size_t(b) * H + h) * N + n;
-
-    float l[MP];
-    uint4 v[MP];
+  for (uint32_t base = warp_base0; base < total; base += U * stride) {
+    float l[U][MP];
+    uint4 v[U][MP];
+    size_t off[U], lrow[U];
+    bool valid[U], lead[U];
 #pragma unroll
-    for (int p = 0; p < MP; ++p) {
-      if (p < parts.n && valid) {
-        l[p] = parts.lse[p][lrow];
-        v[p] = *reinterpret_cast<const uint4*>(parts.o[p] + off);
-      } else {
-        l[p] = -INFINITY;
-        v[p] = make_uint4(0, 0, 0, 0);
+    for (int u = 0; u < U; ++u) {
+      const uint32_t gid = base + u * stride + lane;
+      valid[u] = gid < total;
+      const uint32_t row = valid[u] ? gid / G : 0;  // (b * N + n) * H + h: the memory order of o
+      const uint32_t g = gid - row * G;
+      const uint32_t bn = row / uint32_t(H);
+      const uint32_t h = row - bn * uint32_t(H);
+      const uint32_t b = bn / uint32_t(N);
+      const uint32_t n = bn - b * uint32_t(N);
+      off[u] = size_t(row) * D + g * 8;
+      lrow[u] = (size_t(b) * H + h) * N + n;
+      lead[u] = g == 0;
+#pragma unroll
+      for (int p = 0; p < MP; ++p) {
+        if (p < parts.n && valid[u]) {
+          l[u][p] = parts.lse[p][lrow[u]];
+          v[u][p] = *reinterpret_cast<const uint4*>(parts.o[p] + off[u]);
+        } else {
+          l[u][p] = -INFINITY;
+          v[u][p] = make_uint4(0, 0, 0, 0);
+        }
       }
     }
     __syncwarp();
-    float m = -INFINITY;
 #pragma unroll
-    for (int p = 0; p < MP; ++p) m = fmaxf(m, l[p]);
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    float out_lse = -INFINITY;
-    if (m > -INFINITY) {
-      float w[MP];
-      float tot = 0.f;
-#pragma unroll
-      for (int p = 0; p < MP; ++p) {
-        w[p] = (l[p] > -INFINITY) ? expf(l[p] - m) : 0.f;
-        tot += w[p];
-      }
-      const float inv = 1.f / tot;
-#pragma unroll
-      for (int p = 0; p < MP; ++p) {
-        if (w[p] == 0.f) continue;
-        const float wp = w[p] * inv;
-        const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&v[p]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(x[e]);
-          acc[2 * e] = fmaf(wp, f.x, acc[2 * e]);
-          acc[2 * e + 1] = fmaf(wp, f.y, acc[2 * e + 1]);
-        }
-      }
-      out_lse = m + logf(tot);
-    }
-    if (valid) {
-      uint4 res;
-      uint32_t* r = reinterpret_cast<uint32_t*>(&res);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
-        r[e] = *reinterpret_cast<uint32_t*>(&h2);
-      }
-      *reinterpret_cast<uint4*>(o + off) = res;
-      if (lse && g == 0) lse[lrow] = out_lse;
-    }
+    for (int u = 0; u < U; ++u)
+      if (valid[u]) merge_one<D, MP>(parts, l[u], v[u], o, lse, off[u], lrow[u], lead[u]);
   }
 }
 
