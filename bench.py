@@ -133,9 +133,11 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
 
-    def stop(self):
+    def stop(self, window=None):
+        """Median clocks of the samples under load; with window = (t0, t1) host times, only the
+        samples taken inside it (50 ms of slack at the end for the sampling interval)."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -145,7 +147,11 @@ class ClockSampler:
             self.proc.kill()
         self.thread.join(timeout=2)
         rows = []
-        for ln in self.lines:
+        lines = self.lines
+        if window is not None:
+            inside = [(ts, ln) for ts, ln in lines if window[0] <= ts <= window[1] + 0.05]
+            lines = inside or lines
+        for _, ln in lines:
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 8:
                 continue
@@ -159,7 +165,8 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v.lower() == "active"})
         return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in loaded),
-                "reasons": reasons, "samples": len(loaded)}
+                "reasons": reasons, "samples": len(loaded),
+                "window": "timed region" if window is not None and lines is not self.lines else "whole run"}
 
 
 def live_flop(mask: torch.Tensor, N: int, d: int, tile: int) -> float:
@@ -315,6 +322,9 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     la.load()
 
+    clocks = ClockSampler(local)
+    clocks.start()  # started early: nvidia-smi takes a while to produce its first sample
+
     wl = rank_workload(wlmod.WORKLOADS[args.workload], rank, args.heads)
     B, N, H, d = wl.B, wl.N, wl.H, wl.d
     tile, T, W = la.lite_mask_geometry(N, d)
@@ -336,8 +346,6 @@ def main():
         q, k, v = qkv[t]
         la.lite_attn_fwd(q, k, v, masks[t], masks[t + 1], tau=tau_at(wl, t, args.tau), o=out, lse=out_lse)
 
-    clocks = ClockSampler(local)
-    clocks.start()
     for t in range(args.warmup):
         fwd(t)
     torch.cuda.synchronize()
@@ -352,6 +360,7 @@ def main():
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
+    t_wall0 = time.time()
     start.record()
     for i in range(args.steps):
         la.lite_set_kernel_events(*ev[i])
@@ -359,9 +368,10 @@ def main():
     end.record()
     la.lite_set_kernel_events(None, None)
     torch.cuda.synchronize()
+    t_wall1 = time.time()
     if dist:
         dist.barrier()
-    clock_info = clocks.stop()
+    clock_info = clocks.stop(window=(t_wall0, t_wall1))
     elapsed_ms = max_over_ranks(start.elapsed_time(end), dist, dev)
     status = la.lite_get_device_status()
     assert status == 0, la.status_string(status)
