@@ -393,6 +393,10 @@ __global__ void __launch_bounds__(320, 1)
       const uint64_t q_desc = umma_desc_sw128(sQ, 16, 1024);
       const uint64_t k_desc0 = umma_desc_sw128(sK, 16, 1024);
       const uint64_t v_desc0 = umma_desc_sw128(sV, C::KV_CHUNK, 1024);
+      // shared-memory addresses of the per-buffer barriers (8 bytes apart), computed once
+      const uint32_t bar_kv = BAR(kv_full[0]), bar_s = BAR(s_full[0]);
+      const uint32_t bar_p = BAR(p_full[0]), bar_pv = BAR(pv_done[0]);
+      uint32_t v_stage = 0;  // (t-1) % 3 for the pending PV
       auto issue_pv = [&](uint32_t u) -> bool {
         // the first PV of an item overwrites O_0 / O_1 (the first two, one per accumulator): the
         // previous item's epilogue must have read both (o_free: one phase per item, exact because
@@ -400,18 +404,19 @@ __global__ void __launch_bounds__(320, 1)
         if (pend_idx == 0 && pend_item >= 1 && !wt.wait(BAR(o_free), (pend_item - 1) & 1)) return false;
         LITE_TRACE(1, 3, u);
         // p_full of buffer u%2 next completes for tile u+2, whose S needs QK_{u+2}, issued after this
-        if (!wt.wait(BAR(p_full[u & 1]), (u >> 1) & 1)) return false;
+        if (!wt.wait(bar_p + (u & 1) * 8, (u >> 1) & 1)) return false;
         LITE_TRACE(1, 4, u);
         ptx::tc_fence_after();
         const uint32_t p_tmem = tmem + C::S_COL + (u & 1) * BN;
         const uint32_t o_tmem = tmem + C::O_COL + (u & 1) * D;
-        const uint64_t vd = v_desc0 + uint64_t(((u % 3) * C::KV_BYTES) >> 4);
+        const uint64_t vd = v_desc0 + uint64_t(v_stage * (C::KV_BYTES >> 4));
+        v_stage = v_stage == 2 ? 0 : v_stage + 1;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
           ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + uint64_t(kk * 128), C::IDESC_PV,
                       (pend_idx < 2 && kk == 0) ? 0u : 1u);
         // the epilogue of group u%2 waits for the item's last PV into its accumulator
-        if (pend_idx >= pend_n - 2) ptx::mma_commit(BAR(pv_done[u & 1]));
+        if (pend_idx >= pend_n - 2) ptx::mma_commit(bar_pv + (u & 1) * 8);
         LITE_TRACE(1, 6, u);
         return true;
       };
@@ -442,7 +447,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int idx = 0; idx < it.n && ok; ++idx, ++t) {
           // kv_full of this slot next completes for bundle t+2, loaded after QK_t finished
           LITE_TRACE(1, 0, t);
-          if (!wt.wait(BAR(kv_full[t & 1]), (t >> 1) & 1)) { ok = false; break; }
+          if (!wt.wait(bar_kv + (t & 1) * 8, (t >> 1) & 1)) { ok = false; break; }
           LITE_TRACE(1, 1, t);
           ptx::tc_fence_after();
           const uint64_t kd = k_desc0 + uint64_t(((t & 1) * C::KV_BYTES) >> 4);
@@ -453,7 +458,7 @@ __global__ void __launch_bounds__(320, 1)
             const uint64_t offk = uint64_t((kk >> 2) * (C::KV_CHUNK >> 4) + (kk & 3) * 2);
             ptx::mma_ss(s_tmem, q_desc + off, kd + offk, C::IDESC_QK, kk > 0 ? 1u : 0u);
           }
-          ptx::mma_commit(BAR(s_full[t & 1]));
+          ptx::mma_commit(bar_s + (t & 1) * 8);
           if (idx == it.n - 1) ptx::mma_commit(BAR(q_empty));
           LITE_TRACE(1, 2, t);
           if (t >= 1 && !issue_pv(t - 1)) { ok = false; break; }
