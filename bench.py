@@ -396,6 +396,9 @@ def main():
     dense_ms = sum(a.elapsed_time(b) for a, b in d_ev)
     sparse_ms = elapsed_ms
 
+    # ---- steady state: one fixed mask_in (the last timed step's) re-run with a scratch mask_out
+    steady = run_steady(la, qkv[S - 1], masks[S - 1], tau_at(wl, S - 1, args.tau), N, d, tile, T, dense_flop_step)
+
     # ---- roofline of the attention kernel (executed FLOP per launch / its event-timed duration)
     burst, sustained, peak_src = measured_peaks()
     attn_avg_ms = sum(attn_ms) / len(attn_ms)
@@ -422,7 +425,8 @@ def main():
         q, k, v = qkv[t_mid]
         fl, dt, what = cpu_oracle_sample(q, k, v, masks[t_mid], tau_at(wl, t_mid, args.tau))
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
-               "sample": f"{what}; dense-equivalent FLOP / oracle wall time ({dt:.1f} s)"}
+               "sample": f"{what}; dense-equivalent FLOP / oracle wall time ({dt:.1f} s)",
+               "extrapolated_step_s": dense_flop_step / (fl / dt)}
 
     if rank == 0:
         line = {
@@ -443,6 +447,7 @@ def main():
             "roofline": roofline,
             "gpu_launches": 3 * args.steps,
             "clocks": clock_info,
+            "steady": steady,
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
@@ -450,6 +455,64 @@ def main():
     if dist:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_steady(la, qkv, mask_in, tau, N, d, tile, T, dense_flop, warmup=5, reps=20):
+    """The same layer step repeated with one fixed mask_in into a scratch mask_out (the mask does not
+    grow between repetitions): per-call time of lite_attn_fwd, of its attention kernel, and of the
+    compaction and schedule kernels launched alone on the same mask. Outside the timed region."""
+    q, k, v = qkv
+    B, _, H, _ = q.shape
+    scratch = torch.empty_like(mask_in)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+
+    def call():
+        la.lite_attn_fwd(q, k, v, mask_in, scratch, tau=tau, o=o, lse=lse)
+
+    for _ in range(warmup):
+        call()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ka, kb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ka.record()
+    kb.record()
+    attn = 0.0
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(reps):
+        call()
+    b.record()
+    torch.cuda.synchronize()
+    call_ms = a.elapsed_time(b) / reps
+    la.lite_set_kernel_events(ka, kb)
+    for _ in range(reps):
+        call()
+        torch.cuda.synchronize()
+        attn += ka.elapsed_time(kb)
+    la.lite_set_kernel_events(None, None)
+    # the two preparation kernels alone, through the C ABI with preallocated outputs
+    lib, st = la.load(), torch.cuda.current_stream().cuda_stream
+    lst = torch.empty((B, H, T, T), dtype=torch.int16, device=q.device)
+    counts = torch.empty((B, H, T), dtype=torch.int32, device=q.device)
+    order = torch.empty(B * H * T, dtype=torch.int32, device=q.device)
+
+    def compact():
+        assert lib.lite_mask_to_list(mask_in.data_ptr(), lst.data_ptr(), counts.data_ptr(), B, H, N, d, st) == 0
+
+    def schedule():
+        assert lib.lite_schedule(counts.data_ptr(), order.data_ptr(), B, H, T, st) == 0
+
+    compact()
+    compact_ms = _time_call(compact, reps)
+    schedule_ms = _time_call(schedule, reps)
+    status = la.lite_get_device_status()
+    assert status == 0, la.status_string(status)
+    flop = live_flop(mask_in, N, d, tile)
+    return {"mask": "input mask of the last timed step", "warmup": warmup, "reps": reps,
+            "skipped_tile_fraction": skipped_fraction(mask_in, T), "ms_per_call": call_ms,
+            "dense_equiv_tflops": dense_flop / (call_ms * 1e-3) / 1e12,
+            "executed_tflops": flop / (call_ms * 1e-3) / 1e12,
+            "attn_ms": attn / reps, "compact_ms": compact_ms, "schedule_ms": schedule_ms}
 
 
 def run_e2e(args, la, wl, qkv, masks, dev, world, dist):
