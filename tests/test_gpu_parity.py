@@ -261,6 +261,25 @@ def test_480p_layer_sampled_late_steps():
     assert sp[-1] > 0
 
 
+@pytest.mark.parametrize("d,F,gh,gw", [(64, 27, 133, 73), (128, 5, 47, 2231)])
+def test_maximum_tile_count(d, F, gh, gw):
+    """The largest layer the library accepts: 4096 query and key tiles (N = 262,143 at d=64 and
+    524,285 at d=128, each with a ragged last tile, so list entries reach 4095), a random Skip-Mask
+    and QK-Skip on; sampled query tiles, the last one included, against the oracle."""
+    w = wl.small_workload(1, 1, F, gh, gw, d, steps=1, locality=3.0, tau=-3.0, seed_offset=4096 + d)
+    q, k, v = wl.Trajectory(w, device="cuda").current()
+    tile, T, _ = la.lite_mask_geometry(w.N, d)
+    assert T == 4096 and w.N % tile != 0
+    m_in = wl.random_mask(1, 1, T, 0.8, seed=d).cuda()
+    m_out = torch.empty_like(m_in)
+    o, lse = la.lite_attn_fwd(q, k, v, m_in, m_out, tau=-3.0)
+    assert la.lite_get_device_status() == 0
+    ref = oracle_step(q, k, v, m_in, -3.0, query_tiles=[(0, 0, 0), (0, 0, 2047), (0, 0, T - 1)])
+    rep = compare(o, lse, m_out, ref)
+    assert_within(rep)
+    print(f"d={d} N={w.N} flagged(sampled)={rep.flagged} o_max={rep.o_max_abs:.2e} lse={rep.lse_max_abs:.2e}")
+
+
 def test_720p_layer_sampled():
     _full_size("720p", 2, 8)
 
