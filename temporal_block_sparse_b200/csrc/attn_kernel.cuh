@@ -105,8 +105,14 @@ struct AttnCfg {
   static constexpr int CTL_BYTES = 512;
   static constexpr int OFF_X = OFF_CTL + CTL_BYTES;  // tile-max mailbox float[4][128]; epilogue float[2][2][128]
   static constexpr int X_BYTES = 4 * 128 * 4 + 2 * 2 * 128 * 4;
+  // O staging for the TMA stores of the epilogue: per softmax warp, 16 rows of its group's D/2
+  // columns (D bytes a row; 128-byte swizzled for D = 128, so the region is 1024-aligned)
+  static constexpr int OST_ROWS = 16;
+  static constexpr int OST_WARP = OST_ROWS * D;
+  static constexpr int OFF_OST = (OFF_X + X_BYTES + 1023) / 1024 * 1024;
+  static constexpr int OST_BYTES = 8 * OST_WARP;
   // one CTA per SM: the request is padded so that two never fit (TMEM is sized for one)
-  static constexpr int SMEM_USED = OFF_X + X_BYTES + 1024;
+  static constexpr int SMEM_USED = OFF_OST + OST_BYTES + 1024;
   static constexpr int SMEM_BYTES = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   // TMEM columns: S_0 [0, BN), S_1 [BN, 2BN), O_0 [2BN, 2BN+D), O_1 [2BN+D, 2BN+2D)
   static constexpr uint32_t S_COL = 0;
@@ -247,7 +253,8 @@ __device__ __forceinline__ int key_entry(const AttnParams& p, int row, int idx) 
 template <int D, int BN>
 __global__ void __launch_bounds__(320, 1)
     lite_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                     const AttnParams p) {
   using C = AttnCfg<D, BN>;
   static_assert(sizeof(AttnCtl) <= C::CTL_BYTES, "control block");
   extern __shared__ uint8_t smem_raw[];
@@ -286,6 +293,7 @@ __global__ void __launch_bounds__(320, 1)
     ptx::prefetch_tmap(&tmQ);
     ptx::prefetch_tmap(&tmK);
     ptx::prefetch_tmap(&tmV);
+    ptx::prefetch_tmap(&tmO);
   }
   if constexpr (C::BQ < C::BM) {
     // Q rows past the query tile are never loaded; keep them zero so their S rows stay finite.
@@ -629,7 +637,8 @@ __global__ void __launch_bounds__(320, 1)
         m_true = fmaxf(m_true, loc);
       }
       // epilogue: each group waits for its last PV, the two partial softmaxes are combined,
-      // group g stores columns [g*D/2, (g+1)*D/2) of O (bf16) and group 0 the lse
+      // group g writes columns [g*D/2, (g+1)*D/2) of O (bf16, through shared memory and TMA
+      // stores) and group 0 the lse
       if (first < it.n) {
         wt.wait(BAR(pv_done[grp]), pv_phase & 1);  // one phase per item in which this group has a tile
         ++pv_phase;
@@ -650,28 +659,53 @@ __global__ void __launch_bounds__(320, 1)
       const float lt = a0 * l0 + a1 * l1;
       const float inv_l = 1.f / lt;
       const float w0 = a0 * inv_l, w1 = a1 * inv_l;
-#pragma unroll 1
+      // The group's D/2 columns of O, combined and rounded to bf16, leave through shared memory:
+      // each warp stages the rows of lanes 0-15, then those of lanes 16-31, and its lane 0 issues
+      // one TMA store per half (rows past Nq are clipped by the TMA unit). The threads never wait
+      // for global memory; a staging half is rewritten only after its previous store has read it.
+      uint32_t ow[D / 4];  // this row's D/2 bf16 columns, packed in pairs
+#pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         const int col = grp * (D / 2) + c * 32;
         uint32_t r0[32], r1[32];
         ptx::tmem_ld32(tmem + lane_base + C::O_COL + 0 * D + col, r0);
         ptx::tmem_ld32(tmem + lane_base + C::O_COL + 1 * D + col, r1);
         ptx::tmem_wait_ld();
-        if (valid_row) {
-          uint32_t pk[16];
 #pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            // an accumulator without a partial may hold stale data: select, never multiply by zero
-            const float o0 = (has0 ? w0 * __uint_as_float(r0[2 * x]) : 0.f) +
-                             (has1 ? w1 * __uint_as_float(r1[2 * x]) : 0.f);
-            const float o1 = (has0 ? w0 * __uint_as_float(r0[2 * x + 1]) : 0.f) +
-                             (has1 ? w1 * __uint_as_float(r1[2 * x + 1]) : 0.f);
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(o0, o1);
-            pk[x] = *reinterpret_cast<uint32_t*>(&h2);
+        for (int x = 0; x < 16; ++x) {
+          // an accumulator without a partial may hold stale data: select, never multiply by zero
+          const float o0 = (has0 ? w0 * __uint_as_float(r0[2 * x]) : 0.f) +
+                           (has1 ? w1 * __uint_as_float(r1[2 * x]) : 0.f);
+          const float o1 = (has0 ? w0 * __uint_as_float(r0[2 * x + 1]) : 0.f) +
+                           (has1 ? w1 * __uint_as_float(r1[2 * x + 1]) : 0.f);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(o0, o1);
+          ow[c * 16 + x] = *reinterpret_cast<uint32_t*>(&h2);
+        }
+      }
+      {
+        uint8_t* stage = smem + C::OFF_OST + (grp * 4 + quarter) * C::OST_WARP;
+        const int srow = lane & (C::OST_ROWS - 1);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          if (lane == 0) ptx::bulk_wait_group_read0();
+          __syncwarp();
+          if ((lane >> 4) == half) {
+#pragma unroll
+            for (int x = 0; x < D / 16; ++x) {
+              // 16-byte chunk x of the row; 128-byte swizzle (chunk ^ row % 8) for D = 128
+              const int pc = D == 128 ? (x ^ (srow & 7)) : x;
+              *reinterpret_cast<uint4*>(stage + srow * D + pc * 16) =
+                  make_uint4(ow[4 * x], ow[4 * x + 1], ow[4 * x + 2], ow[4 * x + 3]);
+            }
           }
-          uint4* dst = reinterpret_cast<uint4*>(p.o + o_off * D + col);
-#pragma unroll
-          for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          const int row_in_tile = quarter * 32 + half * C::OST_ROWS;
+          if (lane == 0 && row_in_tile < C::BQ && it.qi * C::BQ + row_in_tile < p.Nq) {
+            ptx::tma_store_5d(&tmO, ptx::smem_addr(stage), grp * (D / 2) % 64, it.qi * C::BQ + row_in_tile,
+                              grp * (D / 2) / 64, it.h, it.b);
+            ptx::bulk_commit_group();
+          }
         }
       }
       if (valid_row && grp == 0 && p.lse)
@@ -680,6 +714,9 @@ __global__ void __launch_bounds__(320, 1)
       ptx::mbar_arrive(BAR(o_free));
       t0 += it.n;
     }
+    // the staged O rows must have been written out before the CTA (and its shared memory) ends
+    if (lane == 0) ptx::bulk_wait_group0();
+    __syncwarp();
   }
 #undef BAR
 

@@ -134,6 +134,20 @@ bool make_tmap(CUtensorMap* map, const void* ptr, int B, int N, int H, int d, in
   return r == CUDA_SUCCESS;
 }
 
+// O as the epilogue stores it: the same 5-D view as q, a box of 16 rows of one softmax group's
+// d/2 columns (64 columns in one 128-byte swizzled panel for d = 128; 32 columns, unswizzled, for
+// d = 64).
+bool make_tmap_o(CUtensorMap* map, void* ptr, int B, int N, int H, int d) {
+  cuuint64_t dims[5] = {64, cuuint64_t(N), cuuint64_t(d / 64), cuuint64_t(H), cuuint64_t(B)};
+  cuuint64_t strides[4] = {cuuint64_t(H) * d * 2, 128, cuuint64_t(d) * 2, cuuint64_t(N) * H * d * 2};
+  cuuint32_t box[5] = {cuuint32_t(d / 2), 16, 1, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, ptr, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 float resolve_scale(float scale, int d) {
   if (!(scale > 0.f) || std::isnan(scale)) return 1.0f / std::sqrt(static_cast<float>(d));
   return scale;
@@ -149,16 +163,16 @@ int launch_attention(DeviceCache* dc, int cfg_slot, const void* q, const void* k
       return LITE_ERR_CUDA;
     dc->smem_set[cfg_slot] = true;
   }
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_tmap(&tq, q, p.B, p.Nq, p.H, D, C::BQ) || !make_tmap(&tk, k, p.B, p.Nk, p.H, D, BN) ||
-      !make_tmap(&tv, v, p.B, p.Nk, p.H, D, BN))
+      !make_tmap(&tv, v, p.B, p.Nk, p.H, D, BN) || !make_tmap_o(&to, p.o, p.B, p.Nq, p.H, D))
     return LITE_ERR_CUDA;
   int grid = dc->sms;
   if (g_opt.max_ctas > 0 && g_opt.max_ctas < grid) grid = g_opt.max_ctas;
   if (p.n_items < grid) grid = p.n_items;
   if (grid <= 0) return LITE_OK;
   if (g_ev_before) cudaEventRecord(g_ev_before, stream);
-  lite::lite_attn_kernel<D, BN><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  lite::lite_attn_kernel<D, BN><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
   if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
   if (g_ev_after) cudaEventRecord(g_ev_after, stream);
   return LITE_OK;
