@@ -132,6 +132,15 @@ struct AttnCfg {
   static_assert(NCHUNK == 1 || (Q_CHUNK == BQ * 128 && KV_CHUNK == BN * 128), "panel strides");
 };
 
+// A work item (one query tile of one head), decoded once by the producer and handed to the other
+// roles through shared memory, with its first two list entries (the first tile of each group).
+struct ItemInfo {
+  int row;     // (b*H + h)*Tq + qi; -1 marks the end of the work
+  int n;       // live key tiles
+  int b, h, qi;
+  int e0, e1;  // list entries 0 and 1 (when n > 0, n > 1)
+};
+
 // Control block in shared memory (barriers are 8-byte mbarrier objects).
 struct alignas(8) AttnCtl {
   uint64_t q_full, q_empty;
@@ -144,7 +153,7 @@ struct alignas(8) AttnCtl {
   uint64_t item_full[2], item_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
-  int item[2];
+  ItemInfo info[2];                  // the handed-out items
   int abort;
   uint32_t tiles;                    // live tiles this CTA processed (measurement hook)
 };
@@ -228,11 +237,7 @@ struct Waiter {
   }
 };
 
-struct ItemInfo {
-  int row;  // (b*H + h)*Tq + qi
-  int n;    // live key tiles
-  int b, h, qi;
-};
+__device__ __forceinline__ int key_entry(const AttnParams& p, int row, int idx);
 
 __device__ __forceinline__ ItemInfo decode_item(const AttnParams& p, int item) {
   ItemInfo it;
@@ -242,6 +247,8 @@ __device__ __forceinline__ ItemInfo decode_item(const AttnParams& p, int item) {
   it.qi = it.row - bh * p.Tq;
   it.b = bh / p.H;
   it.h = bh - it.b * p.H;
+  it.e0 = it.n > 0 ? key_entry(p, it.row, 0) : 0;
+  it.e1 = it.n > 1 ? key_entry(p, it.row, 1) : 0;
   return it;
 }
 
@@ -355,11 +362,12 @@ __global__ void __launch_bounds__(320, 1)
         // dynamic hand-out in schedule order; without a counter, static striding (uniform items)
         int item = p.work_counter ? atomicAdd(p.work_counter, 1) : int(blockIdx.x + items * gridDim.x);
         if (item >= p.n_items) item = -1;
-        ctl->item[slot] = item;
+        ItemInfo it{-1, 0, 0, 0, 0, 0, 0};
+        if (item >= 0) it = decode_item(p, item);
+        ctl->info[slot] = it;
         ptx::mbar_arrive(BAR(item_full[slot]));
         ++items;
         if (item < 0) break;
-        const ItemInfo it = decode_item(p, item);
         if (it.n == 0) continue;
         // Q is read by one item's QKs; q_empty is committed after the item's last QK
         if (qn >= 1) ok = wt.wait(BAR(q_empty), (qn - 1) & 1);
@@ -370,7 +378,8 @@ __global__ void __launch_bounds__(320, 1)
         q_par = qn & 1;
         ++qn;
         for (int idx = 0; idx < it.n && ok; ++idx)
-          ok = bundle(true, key_entry(p, it.row, idx) & kListIndexMask, it.h, it.b);
+          ok = bundle(true, (idx == 0 ? it.e0 : idx == 1 ? it.e1 : key_entry(p, it.row, idx)) & kListIndexMask,
+                      it.h, it.b);
       }
       ctl->tiles = t;
       if (ok && t >= 1) bundle(false, 0, 0, 0);  // V of the last tile
@@ -432,11 +441,10 @@ __global__ void __launch_bounds__(320, 1)
         const int slot = items & 1;
         ok = wt.wait(BAR(item_full[slot]), (items >> 1) & 1);
         if (!ok) break;
-        const int item = ctl->item[slot];
+        const ItemInfo it = ctl->info[slot];
         ptx::mbar_arrive(BAR(item_empty[slot]));
         ++items;
-        if (item < 0) break;
-        const ItemInfo it = decode_item(p, item);
+        if (it.row < 0) break;
         if (it.n == 0) continue;
         if (p.debug_stall && !stalled) {
           // test hook: withhold all work of this item until the softmax warps give up
@@ -500,12 +508,11 @@ __global__ void __launch_bounds__(320, 1)
     while (true) {
       const int slot = items & 1;
       bool ok = wt.wait(BAR(item_full[slot]), (items >> 1) & 1);
-      const int item = ctl->item[slot];
+      const ItemInfo it = ctl->info[slot];
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(BAR(item_empty[slot]));
       ++items;
-      if (!ptx::named_bar_and(3, 256, ok) || item < 0) break;
-      const ItemInfo it = decode_item(p, item);
+      if (!ptx::named_bar_and(3, 256, ok) || it.row < 0) break;
       const int n_row = it.qi * C::BQ + r;
       const bool valid_row = (r < C::BQ) && (n_row < p.Nq);
       const size_t o_off = (size_t(it.b) * p.Nq + n_row) * p.H + it.h;
@@ -522,7 +529,7 @@ __global__ void __launch_bounds__(320, 1)
       float l = 0.f;             // this group's share of the row sum
       // this group's tiles of the item: idx = first, first + 2, ...
       const int first = int((uint32_t(grp) - t0) & 1u);
-      int j_next = first < it.n ? key_entry(p, it.row, first) : 0;
+      int j_next = first < it.n ? (first == 0 ? it.e0 : it.e1) : 0;
       for (int idx = first; idx < it.n; idx += 2) {
         const uint32_t t = t0 + idx;
         const int j = j_next & kListIndexMask;
