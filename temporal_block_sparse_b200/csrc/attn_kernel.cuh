@@ -1,31 +1,33 @@
 // attn_kernel.cuh -- persistent block-sparse attention forward for sm_100a (tcgen05 + TMEM + TMA).
 //
-// One CTA per SM walks a list of work items; an item is one query tile of one (b, h). For an item
-// it streams only the live key tiles of that query tile (LiteAttention README, "Full-Stage
-// Elimination": a skipped tile costs no K/V load, no QK^T, no softmax, no PV), from the highest
-// key-tile index down (README, must_do_list: "we iterate in reverse order inside of the kernel").
-// Queries and keys may differ in length (README, LSE section: partial attentions such as text-to-
-// video over a subset of the keys); a key tile that a must-do range keeps live carries a tag in its
-// list entry and is computed but never flagged.
+// One CTA per SM walks a list of work items; an item is a pair of consecutive query tiles (2i,
+// 2i+1) of one (b, h). For each query tile it computes only the live key tiles of that tile
+// (LiteAttention README, "Full-Stage Elimination": a skipped tile costs no K/V load, no QK^T, no
+// softmax, no PV), from the highest key-tile index down (README, must_do_list: "we iterate in
+// reverse order inside of the kernel"). The two query tiles share K/V: the CTA walks the union of
+// their two Skip-Lists, loads each union tile once, and computes it for the query tiles it is live
+// for. Queries and keys may differ in length (README, LSE section: partial attentions such as
+// text-to-video over a subset of the keys); a key tile that a must-do range keeps live carries a
+// tag in its list entry and is computed but never flagged.
 //
 // Warp roles (320 threads):
-//   warp 0       TMA producer: Q once per item; per live tile K_j into a 2-stage ring and V_j into
-//                a 3-stage ring (separate barriers, so S = QK^T never waits for V).
-//   warp 1       TMEM allocator and single-thread tcgen05 MMA issuer, in the order
-//                QK_0, QK_1, PV_0, QK_2, PV_1, ... over the live tiles of consecutive items:
-//                  S_t = Q K_t^T  (SS form) into TMEM buffer t%2,
-//                  O_{t%2} += P_t V_t (TS form: P read from TMEM, V from shared memory).
-//   warps 2..5   softmax warpgroup 0: the tiles t with t%2 == 0;  warps 6..9: warpgroup 1, t%2 == 1.
-//                One thread per query row (TMEM lane). The two groups work on consecutive tiles at
-//                the same time, each with its own running exponent reference, row sum and O
-//                accumulator; the epilogue combines the two partial softmaxes exactly. Per tile:
-//                row max; the QK-Skip vote (skill page "Lite Attention Temporal Sparse", Core
-//                Concept: a tile whose local max score is far below the cumulative max is
-//                flagged) against the running max over ALL earlier tiles, for which each group
-//                receives the other's tile maxima through a shared-memory mailbox; one atomicOr
-//                per flagged (query tile, key tile); exp2 (a quarter on the FMA pipe); P (bf16)
-//                back into TMEM over the consumed S columns; O rescale when the group's reference
-//                max grew by more than 2^8.
+//   warp 0       TMA producer: per item the pair's two Q tiles; per union tile u a load bundle with
+//                K_u (2-stage ring) and V_{u-1} (2-stage ring), one barrier per bundle. It walks the
+//                two lists and hands the MMA thread, per union tile, which query tiles it is live
+//                for, in a small shared-memory ring written before the bundle is armed.
+//   warp 1       TMEM allocator and single-thread tcgen05 MMA issuer. Per union tile u, for query
+//                tile g = 0, 1: PV_g(u-1) if u-1 was live for g, then QK_g(u) if u is live for g:
+//                  S_g = Q_g K_u^T    (SS form) into TMEM buffer g,
+//                  O_g += P_g V_{u-1} (TS form: P read from TMEM, V from shared memory).
+//   warps 2..5   softmax warpgroup 0, query tile 0 of the pair; warps 6..9: group 1, query tile 1.
+//                One thread per query row (TMEM lane). Per live tile of its query tile: row max;
+//                the QK-Skip vote (skill page "Lite Attention Temporal Sparse", Core Concept: a
+//                tile whose local max score is far below the cumulative max is flagged) against
+//                the running max over the tile's earlier live tiles; one atomicOr per flagged
+//                (query tile, key tile); exp2 (a quarter on the FMA pipe); P (bf16) back into TMEM
+//                over the consumed S columns; O rescale when the reference max grew by more than
+//                kRescaleLog2. The two groups run on the two query tiles at once, so the latency of
+//                one hides the other's.
 //
 // Every wait is bounded by a wall-clock limit; on expiry the kernel records a timeout in the device
 // status word, every role stops, in-flight copies and MMAs are drained, TMEM is freed and the CTA
@@ -52,13 +54,14 @@ struct AttnParams {
   uint32_t* mask_out;       // [B, H, Tq, W] or null (flags not recorded)
   const int16_t* list;      // [B*H*Tq, Tk] live key tiles, descending (null: all tiles, dense)
   const int32_t* counts;    // [B*H*Tq] live counts (null: Tk each)
-  const int32_t* order;     // [B*H*Tq] work order (null: identity)
+  const int32_t* order;     // [n_items] work order over query-tile pairs (null: identity)
   int32_t* work_counter;    // zero before launch; null = static striding over items
   int* status;              // device status word
   int B, H;
   int Nq, Nk;               // query / key tokens (equal for self attention)
   int Tq, Tk, W;            // query tiles, key tiles, mask words per query tile (ceil(Tk / 32))
-  int n_items;              // B * H * Tq
+  int Pq;                   // query-tile pairs per (b, h): ceil(Tq / 2)
+  int n_items;              // B * H * Pq
   float scale_log2;         // softmax scale * log2(e)
   float tau_log2;           // QK-Skip threshold * log2(e)
   int skip_test;            // 1: run the QK-Skip vote and record flags
@@ -86,30 +89,27 @@ struct AttnParams {
 
 template <int D, int BN>
 struct AttnCfg {
-  static constexpr int BM = 128;                 // MMA M = TMEM lanes = query rows of the tile slot
+  static constexpr int BM = 128;                 // MMA M = TMEM lanes = query rows of a tile slot
   static constexpr int BQ = BN;                  // valid query rows per query tile
-  static constexpr int KST = 2;                  // K stages
-  static constexpr int VST = 3;                  // V stages
   static constexpr int THREADS = 320;            // producer warp, MMA warp, 2 softmax warpgroups
   static constexpr int NCHUNK = D / 64;          // 128-byte swizzle atoms along d
-  static constexpr int Q_CHUNK = BM * 128;       // bytes between d-chunks of Q in smem
+  static constexpr int Q_CHUNK = BM * 128;       // bytes between d-chunks of a Q tile in smem
   static constexpr int KV_CHUNK = BN * 128;      // bytes between d-chunks of a K or V tile
-  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int Q_BYTES = BM * D * 2;     // one Q tile slot
   static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr uint32_t Q_TX = BQ * D * 2;   // bytes the Q load delivers
+  static constexpr uint32_t Q_TX = BQ * D * 2;   // bytes one Q load delivers
   static constexpr uint32_t KV_TX = BN * D * 2;  // bytes of one K or V tile
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr int OFF_CTL = OFF_V + VST * KV_BYTES;
+  static constexpr int OFF_Q = 0;                // Q_0, Q_1
+  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;
+  static constexpr int OFF_CTL = OFF_V + 2 * KV_BYTES;
   static constexpr int CTL_BYTES = 512;
-  static constexpr int OFF_X = OFF_CTL + CTL_BYTES;  // tile-max mailbox float[4][128]; epilogue float[2][2][128]
-  static constexpr int X_BYTES = 4 * 128 * 4 + 2 * 2 * 128 * 4;
-  // O staging for the TMA stores of the epilogue: per softmax warp, 16 rows of its group's D/2
-  // columns (D bytes a row; 128-byte swizzled for D = 128, so the region is 1024-aligned)
+  // O staging for the TMA stores of the epilogue: per softmax warp, 16 rows of D columns, as
+  // NCHUNK 128-byte-swizzled panels of 16 x 128 bytes (1024-aligned)
   static constexpr int OST_ROWS = 16;
-  static constexpr int OST_WARP = OST_ROWS * D;
-  static constexpr int OFF_OST = (OFF_X + X_BYTES + 1023) / 1024 * 1024;
+  static constexpr int OST_PANEL = OST_ROWS * 128;
+  static constexpr int OST_WARP = NCHUNK * OST_PANEL;
+  static constexpr int OFF_OST = (OFF_CTL + CTL_BYTES + 1023) / 1024 * 1024;
   static constexpr int OST_BYTES = 8 * OST_WARP;
   // one CTA per SM: the request is padded so that two never fit (TMEM is sized for one)
   static constexpr int SMEM_USED = OFF_OST + OST_BYTES + 1024;
@@ -132,32 +132,41 @@ struct AttnCfg {
   static_assert(NCHUNK == 1 || (Q_CHUNK == BQ * 128 && KV_CHUNK == BN * 128), "panel strides");
 };
 
-// A work item (one query tile of one head), decoded once by the producer and handed to the other
-// roles through shared memory, with its first two list entries (the first tile of each group).
-struct ItemInfo {
-  int row;     // (b*H + h)*Tq + qi; -1 marks the end of the work
-  int n;       // live key tiles
-  int b, h, qi;
-  int e0, e1;  // list entries 0 and 1 (when n > 0, n > 1)
+// A work item as the producer hands it to the softmax warpgroups: the pair's query tiles, their
+// live counts and their first two list entries.
+struct PairInfo {
+  int row0;      // (b*H + h)*Tq + 2*qp, the first query tile's row; -1 marks the end of the work
+  int n[2];      // live key tiles of query tiles 2qp and 2qp+1 (0 when the second does not exist)
+  int b, h, qp;
+  int e[2][2];   // entries 0 and 1 of each query tile's list
 };
+
+// Per union tile, what the producer tells the MMA thread (one 32-bit word in a 4-slot ring).
+constexpr uint32_t kLive0 = 1u, kLive1 = 2u;        // live for query tile 0 / 1
+constexpr uint32_t kFirst0 = 4u, kFirst1 = 8u;      // first live tile of query tile 0 / 1 in the item
+constexpr uint32_t kLast0 = 16u, kLast1 = 32u;      // last live tile of query tile 0 / 1 in the item
+constexpr uint32_t kItemFirst = 64u;                // first union tile of an item
+constexpr uint32_t kItemLast = 128u;                // last union tile of an item
+constexpr uint32_t kEnd = 256u;                     // no more tiles (the bundle carries the last V)
+constexpr int kItemShift = 12;                      // bits 12..31: the item's number in this CTA
 
 // Control block in shared memory (barriers are 8-byte mbarrier objects).
 struct alignas(8) AttnCtl {
-  uint64_t q_full, q_empty;
-  uint64_t kv_full[2];               // load bundle t landed: K_t (stage t%2) and V_{t-1} (stage (t-1)%3)
-  uint64_t s_full[2];                // S_t ready (buffer t%2, one warpgroup each)
-  uint64_t p_full[2];                // P_t written (buffer t%2)
-  uint64_t pv_done[2];               // last PV of group g in an item finished (accumulator g)
-  uint64_t mx_full[4], mx_empty[4];  // row maxima of tile t posted in / read from mailbox slot t%4
-  uint64_t o_free;                   // epilogue has read both O accumulators
+  uint64_t q_full, q_empty;          // the pair's Q tiles landed / read by the item's last QK
+  uint64_t kv_full[2];               // bundle u landed: K_u (stage u%2) and V_{u-1} (stage (u-1)%2)
+  uint64_t kv_free[2];               // the QKs of union tile u (and every MMA before them) finished
+  uint64_t s_full[2];                // S_g ready (one phase per live tile of query tile g)
+  uint64_t p_full[2];                // P_g written (one phase per live tile of query tile g)
+  uint64_t pv_done[2];               // last PV_g of an item finished (accumulator g)
+  uint64_t o_free[2];                // group g's epilogue has read O_g (one phase per item)
   uint64_t item_full[2], item_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
-  ItemInfo info[2];                  // the handed-out items
   int abort;
-  uint32_t tiles;                    // live tiles this CTA processed (measurement hook)
+  uint32_t tiles;                    // live (query tile, key tile) pairs processed (measurement hook)
+  uint32_t ring[4];                  // per union tile u (slot u%4): the flags above
+  PairInfo info[2];                  // handed-out items
 };
-
 // UMMA shared-memory descriptor, 128-byte swizzle (layout type 2, bits 61-63), version 1 (bit 46).
 __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   uint64_t d = 0;
@@ -237,25 +246,51 @@ struct Waiter {
   }
 };
 
-__device__ __forceinline__ int key_entry(const AttnParams& p, int row, int idx);
-
-__device__ __forceinline__ ItemInfo decode_item(const AttnParams& p, int item) {
-  ItemInfo it;
-  it.row = p.order ? p.order[item] : item;
-  it.n = p.counts ? p.counts[it.row] : p.Tk;
-  const int bh = it.row / p.Tq;
-  it.qi = it.row - bh * p.Tq;
-  it.b = bh / p.H;
-  it.h = bh - it.b * p.H;
-  it.e0 = it.n > 0 ? key_entry(p, it.row, 0) : 0;
-  it.e1 = it.n > 1 ? key_entry(p, it.row, 1) : 0;
-  return it;
-}
-
 // idx-th live key tile of a row, with its kListNoFlag tag (dense: Tk-1, Tk-2, ..., untagged)
 __device__ __forceinline__ int key_entry(const AttnParams& p, int row, int idx) {
   return p.list ? int(p.list[size_t(row) * p.Tk + idx]) : (p.Tk - 1 - idx);
 }
+
+// Work item `item` (in hand-out order) decoded: the pair's rows, live counts and first entries.
+__device__ __forceinline__ PairInfo decode_pair(const AttnParams& p, int item) {
+  PairInfo it;
+  const int pair = p.order ? p.order[item] : item;
+  const int bh = pair / p.Pq;
+  it.qp = pair - bh * p.Pq;
+  it.b = bh / p.H;
+  it.h = bh - it.b * p.H;
+  it.row0 = bh * p.Tq + 2 * it.qp;
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    const bool exists = 2 * it.qp + g < p.Tq;
+    it.n[g] = !exists ? 0 : (p.counts ? p.counts[it.row0 + g] : p.Tk);
+    it.e[g][0] = it.n[g] > 0 ? key_entry(p, it.row0 + g, 0) : 0;
+    it.e[g][1] = it.n[g] > 1 ? key_entry(p, it.row0 + g, 1) : 0;
+  }
+  return it;
+}
+
+// Walks one query tile's descending list; the entry after the current one is kept prefetched.
+struct ListCursor {
+  int row, n, i;
+  int cur, nxt;  // raw entries i and i+1
+  __device__ __forceinline__ int head() const { return i < n ? (cur & kListIndexMask) : -1; }
+  __device__ __forceinline__ void advance(const AttnParams& p) {
+    ++i;
+    cur = nxt;
+    if (i + 1 < n) nxt = key_entry(p, row, i + 1);
+  }
+};
+
+// Lazy rescale: the exponent reference of a row moves only when a tile's max exceeds it by more
+// than this many log2 units, so P stays below 2^kRescaleLog2. Measured on this B200: a larger
+// threshold rescales O less often, but P values far above 1 in a single long accumulation raise
+// the output error (8 gives ~15% more RMS error than 0); 2 keeps the error at the level of an
+// exact running max within ~1% of the speed of 8.
+constexpr float kRescaleLog2 = 2.0f;
+
+// Item parity and "not the CTA's first item" travel in the ring word next to the tile flags.
+constexpr uint32_t kItemOdd = 512u, kItemAfterFirst = 1024u;
 
 template <int D, int BN>
 __global__ void __launch_bounds__(320, 1)
@@ -267,8 +302,6 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   AttnCtl* ctl = reinterpret_cast<AttnCtl*>(smem + C::OFF_CTL);
-  float* mailbox = reinterpret_cast<float*>(smem + C::OFF_X);    // [4][128] tile row maxima
-  float* epi = mailbox + 4 * 128;                                // [2 groups][2 values][128]
   const uint32_t sQ = ptx::smem_addr(smem + C::OFF_Q);
   const uint32_t sK = ptx::smem_addr(smem + C::OFF_K);
   const uint32_t sV = ptx::smem_addr(smem + C::OFF_V);
@@ -283,17 +316,14 @@ __global__ void __launch_bounds__(320, 1)
     ptx::mbar_init(BAR(q_empty), 1);
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(BAR(kv_full[b]), 1);
+      ptx::mbar_init(BAR(kv_free[b]), 1);
       ptx::mbar_init(BAR(s_full[b]), 1);
       ptx::mbar_init(BAR(p_full[b]), 128);
       ptx::mbar_init(BAR(pv_done[b]), 1);
+      ptx::mbar_init(BAR(o_free[b]), 128);
       ptx::mbar_init(BAR(item_full[b]), 1);
-      ptx::mbar_init(BAR(item_empty[b]), 9);  // MMA thread + one lane of each softmax warp
+      ptx::mbar_init(BAR(item_empty[b]), 8);  // one lane of each softmax warp
     }
-    for (int b = 0; b < 4; ++b) {
-      ptx::mbar_init(BAR(mx_full[b]), 128);
-      ptx::mbar_init(BAR(mx_empty[b]), 128);
-    }
-    ptx::mbar_init(BAR(o_free), 256);
     ptx::mbar_init(BAR(drain), 1);
     ctl->abort = 0;
     ptx::fence_mbar_init();
@@ -304,10 +334,11 @@ __global__ void __launch_bounds__(320, 1)
   }
   if constexpr (C::BQ < C::BM) {
     // Q rows past the query tile are never loaded; keep them zero so their S rows stay finite.
-    for (int c = 0; c < C::NCHUNK; ++c) {
-      uint4* z = reinterpret_cast<uint4*>(smem + C::OFF_Q + c * C::Q_CHUNK + C::BQ * 128);
-      for (int x = threadIdx.x; x < (C::BM - C::BQ) * 128 / 16; x += blockDim.x) z[x] = make_uint4(0, 0, 0, 0);
-    }
+    for (int g = 0; g < 2; ++g)
+      for (int c = 0; c < C::NCHUNK; ++c) {
+        uint4* z = reinterpret_cast<uint4*>(smem + C::OFF_Q + g * C::Q_BYTES + c * C::Q_CHUNK + C::BQ * 128);
+        for (int x = threadIdx.x; x < (C::BM - C::BQ) * 128 / 16; x += blockDim.x) z[x] = make_uint4(0, 0, 0, 0);
+      }
     ptx::fence_proxy_async_smem();
   }
   if (warp == 1) {
@@ -320,39 +351,43 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = ctl->tmem_base;
   const Waiter wt{&ctl->abort, p.status, p.wait_limit_ns};
 
-  // Barrier phases: t counts the live tiles of all items this CTA processes, in processing order.
-  // Tile t uses S buffer, P slot, accumulator and softmax warpgroup t%2, K stage t%2, V stage t%3,
-  // mailbox slot t%4. Every waiter either observes each phase of a barrier in order, or is
-  // guaranteed by the order of the MMA thread's commits that the barrier is at most one phase
-  // away from the awaited one, so the parity waits are exact.
+  // Barrier phases. Union tiles u are numbered over all items this CTA processes; bundle u uses
+  // kv_full / kv_free slot u%2 and ring slot u%4. s_full[g] and p_full[g] complete once per live
+  // tile of query tile g, q_full / q_empty and o_free[g] once per item with tiles, pv_done[g] once
+  // per item in which query tile g has a live tile. Every waiter either observes each phase of a
+  // barrier in order, or the order of the MMA thread's commits keeps the barrier within one phase
+  // of the awaited one (the argument is written at each wait), so the parity waits are exact.
   if (warp == 0) {
     // ------------------------------------------------------------------------- TMA producer
-    // Load bundle t carries K_t (stage t%2, last read by QK_{t-2}) and V_{t-1} (stage (t-1)%3, last
-    // read by PV_{t-4}, which the MMA thread issues before QK_{t-2}); one wait for QK_{t-2} frees
-    // both, and the MMA thread waits once per tile for the bundle. Bundles follow the CTA's tile
-    // sequence across items; one last bundle carries only the final V.
+    // Bundle u carries K_u (stage u%2) and V_{u-1} (stage (u-1)%2). K stage u%2 was last read by
+    // the QKs of union tile u-2; V stage (u-1)%2 by the PVs of union tile u-3, which the MMA thread
+    // issues before those QKs. So one wait (kv_free of u-2) frees both, and the MMA thread waits
+    // once per union tile. A last bundle carries only the final V, with the end mark.
     if (lane == 0) {
-      uint32_t t = 0, items = 0, qn = 0;
+      uint32_t u = 0, items = 0, qn = 0, live_pairs = 0;
       bool ok = true;
       // last armed phase of each full barrier, so that every issued load can be drained at exit
       bool q_armed = false, kv_armed[2] = {false, false};
       uint32_t q_par = 0, kv_par[2] = {0, 0};
-      int pj = 0, ph = 0, pb = 0;  // coordinates of tile t-1
-      // s_full of buffer t%2 next completes with QK_t, which needs this bundle: the wait is exact
-      auto bundle = [&](bool with_k, int j, int h, int b) -> bool {
-        LITE_TRACE(0, 0, t);
-        if (t >= 2 && !wt.wait(BAR(s_full[t & 1]), ((t - 2) >> 1) & 1)) return false;
-        const uint32_t bar = BAR(kv_full[t & 1]);
-        ptx::mbar_arrive_expect_tx(bar, (with_k ? C::KV_TX : 0u) + (t >= 1 ? C::KV_TX : 0u));
-        if (with_k) ptx::tma_load_5d(sK + (t & 1) * C::KV_BYTES, &tmK, bar, 0, j * BN, 0, h, b);
-        if (t >= 1) ptx::tma_load_5d(sV + ((t - 1) % 3) * C::KV_BYTES, &tmV, bar, 0, pj * BN, 0, ph, pb);
-        kv_armed[t & 1] = true;
-        kv_par[t & 1] = (t >> 1) & 1;
-        LITE_TRACE(0, 1, t);
+      int pj = 0, ph = 0, pb = 0;  // coordinates of union tile u-1
+      // kv_free of slot u%2 next completes with the QKs of union tile u, which need this bundle
+      auto bundle = [&](bool with_k, int j, int h, int b, uint32_t flags) -> bool {
+        LITE_TRACE(0, 0, u);
+        if (u >= 2 && !wt.wait(BAR(kv_free[u & 1]), ((u - 2) >> 1) & 1)) return false;
+        // the ring word is written before the bundle's barrier is armed (release), and read by the
+        // MMA thread after it waited on that barrier (acquire)
+        ctl->ring[u & 3] = flags;
+        const uint32_t bar = BAR(kv_full[u & 1]);
+        ptx::mbar_arrive_expect_tx(bar, (with_k ? C::KV_TX : 0u) + (u >= 1 ? C::KV_TX : 0u));
+        if (with_k) ptx::tma_load_5d(sK + (u & 1) * C::KV_BYTES, &tmK, bar, 0, j * BN, 0, h, b);
+        if (u >= 1) ptx::tma_load_5d(sV + ((u - 1) & 1) * C::KV_BYTES, &tmV, bar, 0, pj * BN, 0, ph, pb);
+        kv_armed[u & 1] = true;
+        kv_par[u & 1] = (u >> 1) & 1;
+        LITE_TRACE(0, 1, u);
         pj = j;
         ph = h;
         pb = b;
-        ++t;
+        ++u;
         return true;
       };
       while (ok) {
@@ -362,27 +397,47 @@ __global__ void __launch_bounds__(320, 1)
         // dynamic hand-out in schedule order; without a counter, static striding (uniform items)
         int item = p.work_counter ? atomicAdd(p.work_counter, 1) : int(blockIdx.x + items * gridDim.x);
         if (item >= p.n_items) item = -1;
-        ItemInfo it{-1, 0, 0, 0, 0, 0, 0};
-        if (item >= 0) it = decode_item(p, item);
+        PairInfo it{};
+        it.row0 = -1;
+        if (item >= 0) it = decode_pair(p, item);
         ctl->info[slot] = it;
         ptx::mbar_arrive(BAR(item_full[slot]));
         ++items;
         if (item < 0) break;
-        if (it.n == 0) continue;
-        // Q is read by one item's QKs; q_empty is committed after the item's last QK
+        if (it.n[0] + it.n[1] == 0) continue;
+        // the pair's Q tiles; q_empty is committed after the item's last QK
         if (qn >= 1) ok = wt.wait(BAR(q_empty), (qn - 1) & 1);
         if (!ok) break;
-        ptx::mbar_arrive_expect_tx(BAR(q_full), C::Q_TX);
-        ptx::tma_load_5d(sQ, &tmQ, BAR(q_full), 0, it.qi * C::BQ, 0, it.h, it.b);
+        ptx::mbar_arrive_expect_tx(BAR(q_full), (it.n[0] > 0 ? C::Q_TX : 0u) + (it.n[1] > 0 ? C::Q_TX : 0u));
+        for (int g = 0; g < 2; ++g)
+          if (it.n[g] > 0)
+            ptx::tma_load_5d(sQ + g * C::Q_BYTES, &tmQ, BAR(q_full), 0, (2 * it.qp + g) * C::BQ, 0, it.h, it.b);
         q_armed = true;
         q_par = qn & 1;
+        // the union of the two descending lists, highest key tile first
+        ListCursor c0{it.row0, it.n[0], 0, it.e[0][0], it.e[0][1]};
+        ListCursor c1{it.row0 + 1, it.n[1], 0, it.e[1][0], it.e[1][1]};
+        const uint32_t item_bits = ((qn & 1) ? kItemOdd : 0u) | (qn >= 1 ? kItemAfterFirst : 0u);
+        uint32_t f = kItemFirst;
+        while (ok) {
+          const int h0 = c0.head(), h1 = c1.head();
+          const int j = max(h0, h1);
+          f |= item_bits;
+          if (h0 == j) f |= kLive0 | (c0.i == 0 ? kFirst0 : 0u) | (c0.i == c0.n - 1 ? kLast0 : 0u);
+          if (h1 == j) f |= kLive1 | (c1.i == 0 ? kFirst1 : 0u) | (c1.i == c1.n - 1 ? kLast1 : 0u);
+          if (h0 == j) c0.advance(p);
+          if (h1 == j) c1.advance(p);
+          const bool last = c0.head() < 0 && c1.head() < 0;
+          if (last) f |= kItemLast;
+          ok = bundle(true, j, it.h, it.b, f);
+          if (last) break;
+          f = 0u;
+        }
+        live_pairs += uint32_t(it.n[0] + it.n[1]);
         ++qn;
-        for (int idx = 0; idx < it.n && ok; ++idx)
-          ok = bundle(true, (idx == 0 ? it.e0 : idx == 1 ? it.e1 : key_entry(p, it.row, idx)) & kListIndexMask,
-                      it.h, it.b);
       }
-      ctl->tiles = t;
-      if (ok && t >= 1) bundle(false, 0, 0, 0);  // V of the last tile
+      ctl->tiles = live_pairs;
+      if (ok) bundle(false, 0, 0, 0, kEnd);  // the last union tile's V, and the end mark
       // Drain: every issued TMA load has landed before this thread leaves (no other thread arms these
       // barriers, so the last armed phase is the one to wait for).
       if (q_armed) wt.wait_drain(BAR(q_full), q_par);
@@ -392,105 +447,93 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------------- MMA issuer
-    // One thread issues, over the CTA's tile sequence (continuously across items):
-    //   QK_t:      S_{t%2} = Q K_t^T          after load bundle t (K_t, V_{t-1}) landed
-    //   PV_{t-1}:  O_{(t-1)%2} += P_{t-1} V_{t-1}   after the softmax released P_{t-1}
-    // Per tile that is two waits, two fences and one commit; the softmax releases P well ahead of
-    // this point, so the waits rarely block. QK_{t+2} reuses S buffer t%2 after PV_t read P_t from
-    // it: MMAs of this thread run in issue order.
+    // Per union tile u, once bundle u landed: for g = 0, 1, PV_g(u-1) if u-1 was live for query
+    // tile g, then QK_g(u) if u is live for it. QK_g(u) reuses S buffer g after PV_g(u-1) read the
+    // P in it, and the next QK_g needs the softmax's P_g of this tile first: MMAs of this thread
+    // run in issue order. One commit per union tile frees the bundle's stages.
     if (lane == 0) {
-      uint32_t t = 0, items = 0, qn = 0;
+      uint32_t u = 0;
+      uint32_t pc[2] = {0, 0};  // P phases consumed per query tile
+      uint32_t prev = 0;        // flags of union tile u-1
       bool ok = true;
-      bool stalled = false;
-      // the tile whose PV is pending: its item number, index in the item and the item's tile count
-      uint32_t pend_item = 0;
-      int pend_idx = 0, pend_n = 0;
       // 128B-swizzled K-major operands advance 32 bytes (>> 4 = 2) per K=16 step inside an atom;
       // V (MN-major) advances 16 rows = 2048 bytes (>> 4 = 128) per step.
-      const uint64_t q_desc = umma_desc_sw128(sQ, 16, 1024);
+      const uint64_t q_desc0 = umma_desc_sw128(sQ, 16, 1024);
       const uint64_t k_desc0 = umma_desc_sw128(sK, 16, 1024);
       const uint64_t v_desc0 = umma_desc_sw128(sV, C::KV_CHUNK, 1024);
-      // shared-memory addresses of the per-buffer barriers (8 bytes apart), computed once
-      const uint32_t bar_kv = BAR(kv_full[0]), bar_s = BAR(s_full[0]);
-      const uint32_t bar_p = BAR(p_full[0]), bar_pv = BAR(pv_done[0]);
-      uint32_t v_stage = 0;  // (t-1) % 3 for the pending PV
-      auto issue_pv = [&](uint32_t u) -> bool {
-        // the first PV of an item overwrites O_0 / O_1 (the first two, one per accumulator): the
-        // previous item's epilogue must have read both (o_free: one phase per item, exact because
-        // the next phase needs this item's PVs)
-        if (pend_idx == 0 && pend_item >= 1 && !wt.wait(BAR(o_free), (pend_item - 1) & 1)) return false;
-        LITE_TRACE(1, 3, u);
-        // p_full of buffer u%2 next completes for tile u+2, whose S needs QK_{u+2}, issued after this
-        if (!wt.wait(bar_p + (u & 1) * 8, (u >> 1) & 1)) return false;
-        LITE_TRACE(1, 4, u);
-        ptx::tc_fence_after();
-        const uint32_t p_tmem = tmem + C::S_COL + (u & 1) * BN;
-        const uint32_t o_tmem = tmem + C::O_COL + (u & 1) * D;
-        const uint64_t vd = v_desc0 + uint64_t(v_stage * (C::KV_BYTES >> 4));
-        v_stage = v_stage == 2 ? 0 : v_stage + 1;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + uint64_t(kk * 128), C::IDESC_PV,
-                      (pend_idx < 2 && kk == 0) ? 0u : 1u);
-        // the epilogue of group u%2 waits for the item's last PV into its accumulator
-        if (pend_idx >= pend_n - 2) ptx::mma_commit(bar_pv + (u & 1) * 8);
-        LITE_TRACE(1, 6, u);
-        return true;
-      };
-      while (ok) {
-        const int slot = items & 1;
-        ok = wt.wait(BAR(item_full[slot]), (items >> 1) & 1);
-        if (!ok) break;
-        const ItemInfo it = ctl->info[slot];
-        ptx::mbar_arrive(BAR(item_empty[slot]));
-        ++items;
-        if (it.row < 0) break;
-        if (it.n == 0) continue;
-        if (p.debug_stall && !stalled) {
-          // test hook: withhold all work of this item until the softmax warps give up
-          stalled = true;
-          const uint64_t s0 = ptx::globaltimer();
-          while (!ctl->abort && ptx::globaltimer() - s0 < 4ull * p.wait_limit_ns) {
-          }
-          if (!ctl->abort) wt.give_up();
-          ok = false;
-          break;
+      const uint32_t bar_kv = BAR(kv_full[0]), bar_free = BAR(kv_free[0]);
+      if (p.debug_stall) {
+        // test hook: withhold all work until the other roles give up
+        const uint64_t s0 = ptx::globaltimer();
+        while (!ctl->abort && ptx::globaltimer() - s0 < 4ull * p.wait_limit_ns) {
         }
-        // q_full completes once per item; the next load waits for this item's q_empty commit
-        ok = wt.wait(BAR(q_full), qn & 1);
-        if (!ok) break;
-        ptx::tc_fence_after();
-        for (int idx = 0; idx < it.n && ok; ++idx, ++t) {
-          // kv_full of this slot next completes for bundle t+2, loaded after QK_t finished
-          LITE_TRACE(1, 0, t);
-          if (!wt.wait(bar_kv + (t & 1) * 8, (t >> 1) & 1)) { ok = false; break; }
-          LITE_TRACE(1, 1, t);
-          ptx::tc_fence_after();
-          const uint64_t kd = k_desc0 + uint64_t(((t & 1) * C::KV_BYTES) >> 4);
-          const uint32_t s_tmem = tmem + C::S_COL + (t & 1) * BN;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = uint64_t((kk >> 2) * (C::Q_CHUNK >> 4) + (kk & 3) * 2);
-            const uint64_t offk = uint64_t((kk >> 2) * (C::KV_CHUNK >> 4) + (kk & 3) * 2);
-            ptx::mma_ss(s_tmem, q_desc + off, kd + offk, C::IDESC_QK, kk > 0 ? 1u : 0u);
-          }
-          ptx::mma_commit(bar_s + (t & 1) * 8);
-          if (idx == it.n - 1) ptx::mma_commit(BAR(q_empty));
-          LITE_TRACE(1, 2, t);
-          if (t >= 1 && !issue_pv(t - 1)) { ok = false; break; }
-          pend_item = qn;
-          pend_idx = idx;
-          pend_n = it.n;
-        }
-        ++qn;
+        if (!ctl->abort) wt.give_up();
+        ok = false;
       }
-      // the last tile's PV, once the final bundle (its V) has landed
-      if (ok && t >= 1) {
-        ok = wt.wait(BAR(kv_full[t & 1]), (t >> 1) & 1);
-        if (ok) {
-          ptx::tc_fence_after();
-          issue_pv(t - 1);
+      while (ok) {
+        // kv_full of slot u%2 next completes for bundle u+2, loaded after the QKs of u finished
+        LITE_TRACE(1, 0, u);
+        if (!wt.wait(bar_kv + (u & 1) * 8, (u >> 1) & 1)) break;
+        LITE_TRACE(1, 1, u);
+        const uint32_t f = ctl->ring[u & 3];
+        ptx::tc_fence_after();
+        // q_full completes once per item; the next load waits for this item's q_empty commit
+        bool need_q = (f & kItemFirst) != 0u;
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          if (prev & (kLive0 << g)) {
+            // The first PV of query tile g in an item overwrites O_g: the previous item's epilogue
+            // of group g must have read it (o_free[g]: one phase per item, exact because the next
+            // phase needs this item's PVs). p_full[g] next completes for g's next live tile, whose
+            // S needs a QK issued after this PV.
+            if ((prev & (kFirst0 << g)) && (prev & kItemAfterFirst) &&
+                !wt.wait(BAR(o_free[g]), (prev & kItemOdd) ? 0u : 1u)) {
+              ok = false;
+              break;
+            }
+            if (!wt.wait(BAR(p_full[g]), pc[g] & 1)) {
+              ok = false;
+              break;
+            }
+            ++pc[g];
+            ptx::tc_fence_after();
+            const uint32_t p_tmem = tmem + C::S_COL + g * BN;
+            const uint32_t o_tmem = tmem + C::O_COL + g * D;
+            const uint64_t vd = v_desc0 + uint64_t((((u - 1) & 1) * C::KV_BYTES) >> 4);
+            const bool fresh = (prev & (kFirst0 << g)) != 0u;
+#pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk)
+              ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + uint64_t(kk * 128), C::IDESC_PV, (fresh && kk == 0) ? 0u : 1u);
+            // the epilogue of group g waits for the item's last PV into its accumulator
+            if (prev & (kLast0 << g)) ptx::mma_commit(BAR(pv_done[g]));
+          }
+          if (f & (kLive0 << g)) {
+            if (need_q) {
+              if (!wt.wait(BAR(q_full), (f & kItemOdd) ? 1u : 0u)) {
+                ok = false;
+                break;
+              }
+              ptx::tc_fence_after();
+              need_q = false;
+            }
+            const uint64_t qd = q_desc0 + uint64_t((g * C::Q_BYTES) >> 4);
+            const uint64_t kd = k_desc0 + uint64_t(((u & 1) * C::KV_BYTES) >> 4);
+            const uint32_t s_tmem = tmem + C::S_COL + g * BN;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t off = uint64_t((kk >> 2) * (C::Q_CHUNK >> 4) + (kk & 3) * 2);
+              const uint64_t offk = uint64_t((kk >> 2) * (C::KV_CHUNK >> 4) + (kk & 3) * 2);
+              ptx::mma_ss(s_tmem, qd + off, kd + offk, C::IDESC_QK, kk > 0 ? 1u : 0u);
+            }
+            ptx::mma_commit(BAR(s_full[g]));
+          }
         }
+        LITE_TRACE(1, 2, u);
+        if (!ok || (f & kEnd)) break;
+        ptx::mma_commit(bar_free + (u & 1) * 8);
+        if (f & kItemLast) ptx::mma_commit(BAR(q_empty));
+        prev = f;
+        ++u;
       }
       // all issued tensor-core work must finish before TMEM is released
       ptx::mma_commit(BAR(drain));
@@ -499,44 +542,51 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------------------- softmax warpgroups
-    const int grp = (warp - 2) >> 2;                // tiles t with t % 2 == grp
+    const int grp = (warp - 2) >> 2;                // query tile 2qp + grp of each pair
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;              // TMEM lane = row inside the tile slot
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
-    const uint32_t vote_bar = 1 + grp;              // named barrier of this warpgroup (128 threads)
-    uint32_t t0 = 0, items = 0, pv_phase = 0;
+    const uint32_t gbar = 1 + grp;                  // named barrier of this warpgroup (128 threads)
+    uint8_t* stage = smem + C::OFF_OST + (grp * 4 + quarter) * C::OST_WARP;
+    uint32_t tg = 0, items = 0, pv_phase = 0;
     while (true) {
       const int slot = items & 1;
       bool ok = wt.wait(BAR(item_full[slot]), (items >> 1) & 1);
-      const ItemInfo it = ctl->info[slot];
+      const PairInfo it = ctl->info[slot];
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(BAR(item_empty[slot]));
       ++items;
-      if (!ptx::named_bar_and(3, 256, ok) || it.row < 0) break;
-      const int n_row = it.qi * C::BQ + r;
-      const bool valid_row = (r < C::BQ) && (n_row < p.Nq);
+      if (!ptx::named_bar_and(gbar, 128, ok) || it.row0 < 0) break;
+      const int qi = 2 * it.qp + grp;
+      const int n = it.n[grp];
+      const int row = it.row0 + grp;
+      const int n_row = qi * C::BQ + r;
+      const bool valid_row = qi < p.Tq && r < C::BQ && n_row < p.Nq;
       const size_t o_off = (size_t(it.b) * p.Nq + n_row) * p.H + it.h;
-      if (it.n == 0) {
+      const bool any = it.n[0] + it.n[1] > 0;
+      if (n == 0) {
+        // a query tile without live key tiles: O = 0, lse = -inf; o_free keeps one phase per item
         if (valid_row) {
-          uint4* dst = reinterpret_cast<uint4*>(p.o + o_off * D + grp * (D / 2));
-          for (int x = 0; x < D / 16; ++x) dst[x] = make_uint4(0, 0, 0, 0);
-          if (p.lse && grp == 0) p.lse[(size_t(it.b) * p.H + it.h) * p.Nq + n_row] = -INFINITY;
+          uint4* dst = reinterpret_cast<uint4*>(p.o + o_off * D);
+          for (int x = 0; x < D / 8; ++x) dst[x] = make_uint4(0, 0, 0, 0);
+          if (p.lse) p.lse[(size_t(it.b) * p.H + it.h) * p.Nq + n_row] = -INFINITY;
         }
+        if (any) ptx::mbar_arrive(BAR(o_free[grp]));
         continue;
       }
-      float m_true = -INFINITY;  // running max over all earlier tiles of the item (log2 units)
-      float m_used = -INFINITY;  // this group's exponent reference (lazy rescale)
-      float l = 0.f;             // this group's share of the row sum
-      // this group's tiles of the item: idx = first, first + 2, ...
-      const int first = int((uint32_t(grp) - t0) & 1u);
-      int j_next = first < it.n ? (first == 0 ? it.e0 : it.e1) : 0;
-      for (int idx = first; idx < it.n; idx += 2) {
-        const uint32_t t = t0 + idx;
-        const int j = j_next & kListIndexMask;
-        const bool may_flag = !(j_next & kListNoFlag);
-        if (idx + 2 < it.n) j_next = key_entry(p, it.row, idx + 2);  // prefetch
+      float m_true = -INFINITY;  // running max over the tile's earlier live key tiles (log2 units)
+      float m_used = -INFINITY;  // exponent reference (lazy rescale)
+      float l = 0.f;             // row sum relative to m_used
+      int e_cur = it.e[grp][0], e_nxt = it.e[grp][1];
+      for (int idx = 0; idx < n; ++idx) {
+        const uint32_t t = tg + idx;
+        const int j = e_cur & kListIndexMask;
+        const bool may_flag = !(e_cur & kListNoFlag);
+        e_cur = e_nxt;
+        if (idx + 2 < n) e_nxt = key_entry(p, row, idx + 2);  // prefetch
         if (r == 0) LITE_TRACE(2 + grp, 0, t);
-        wt.wait(BAR(s_full[grp]), (t >> 1) & 1);
+        // s_full[g] next completes for g's next live tile, whose QK follows this tile's PV
+        wt.wait(BAR(s_full[grp]), t & 1);
         __syncwarp();
         ptx::tc_fence_after();
         const uint32_t s_tmem = tmem + lane_base + C::S_COL + grp * BN;
@@ -566,19 +616,17 @@ __global__ void __launch_bounds__(320, 1)
           m3 = ptx::fmax3(m3, s[x + 6], s[x + 7]);
         }
         const float loc = ptx::fmax3(m0, m1, fmaxf(m2, m3)) * p.scale_log2;
-        if (r == 0) LITE_TRACE(2 + grp, 2, t);
-        // lazy rescale of this group's accumulator: move the reference only when the tile max
-        // exceeds it by more than 8 (log2 units). The previous PV into this accumulator (tile t-2)
-        // was issued before QK_t, so it has completed now that S_t is ready; the rescaled O is
-        // stored before any P of this tile is released to the MMA thread.
-        const bool need = loc > m_used + 8.0f;
+        // lazy rescale of the accumulator: move the reference only when the tile max exceeds it by
+        // more than kRescaleLog2. The previous PV into O_g was issued before this tile's QK, so it
+        // has completed now that S is ready; the rescaled O is stored before P is released.
+        const bool need = loc > m_used + kRescaleLog2;
         float alpha = 1.f;
         if (need) {
           alpha = ptx::ex2(m_used - loc);
           m_used = loc;
           l *= alpha;
         }
-        if (__any_sync(0xffffffffu, need) && idx >= 2) {
+        if (__any_sync(0xffffffffu, need) && idx >= 1) {
           const uint32_t o_tmem = tmem + lane_base + C::O_COL + grp * D;
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
@@ -613,84 +661,46 @@ __global__ void __launch_bounds__(320, 1)
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive(BAR(p_full[grp]));
-        if (r == 0) LITE_TRACE(2 + grp, 6, t);
-        // Post this tile's row maxima for the group that takes tile t+1; they enter its QK-Skip
-        // running max, which its vote reads after its own P release, so the post is off the path
-        // from S to P here too. Slot t%4 is refilled every four tiles, after its reader took tile t-4's.
-        if (t >= 4) wt.wait(BAR(mx_empty[t & 3]), ((t >> 2) - 1) & 1);
-        mailbox[(t & 3) * 128 + r] = loc;
-        ptx::mbar_arrive(BAR(mx_full[t & 3]));
-        if (r == 0) LITE_TRACE(2 + grp, 7, t);
+        if (r == 0) LITE_TRACE(2 + grp, 2, t);
         const float2 acc2 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
         l += acc2.x + acc2.y;
-        // QK-Skip vote, off the path from S to P. The running max over the tiles visited before t
-        // takes in tile t-1's maxima from the other group; every posted slot is consumed (also at
-        // the first tile of an item, where the value is not used) so that the slots stay in step.
-        if (t >= 1) {
-          wt.wait(BAR(mx_full[(t - 1) & 3]), ((t - 1) >> 2) & 1);
-          const float prev = mailbox[((t - 1) & 3) * 128 + r];
-          ptx::mbar_arrive(BAR(mx_empty[(t - 1) & 3]));
-          if (idx > 0) m_true = fmaxf(m_true, prev);
+        if (p.skip_test) {
+          // QK-Skip, off the path from S to P: flag key tile j when loc - m < tau for every valid
+          // row, m the running max over the tile's earlier live key tiles
+          const bool pred = !valid_row || (loc - m_true < p.tau_log2);
+          const bool flag = ptx::named_bar_and(gbar, 128, pred);
+          if (flag && may_flag && r == 0 && p.mask_out && !ctl->abort)
+            atomicOr(p.mask_out + size_t(row) * p.W + (j >> 5), 1u << (j & 31));
         }
         if (r == 0) LITE_TRACE(2 + grp, 3, t);
-        if (p.skip_test) {
-          // QK-Skip: flag tile j when loc - m < tau for every valid row (m over earlier tiles)
-          const bool pred = !valid_row || (loc - m_true < p.tau_log2);
-          const bool flag = ptx::named_bar_and(vote_bar, 128, pred);
-          if (flag && may_flag && r == 0 && p.mask_out && !ctl->abort)
-            atomicOr(p.mask_out + size_t(it.row) * p.W + (j >> 5), 1u << (j & 31));
-        }
-        if (r == 0) LITE_TRACE(2 + grp, 4, t);
         m_true = fmaxf(m_true, loc);
       }
-      // epilogue: each group waits for its last PV, the two partial softmaxes are combined,
-      // group g writes columns [g*D/2, (g+1)*D/2) of O (bf16, through shared memory and TMA
-      // stores) and group 0 the lse
-      if (first < it.n) {
-        wt.wait(BAR(pv_done[grp]), pv_phase & 1);  // one phase per item in which this group has a tile
-        ++pv_phase;
-      }
-      epi[(grp * 2 + 0) * 128 + r] = m_used;
-      epi[(grp * 2 + 1) * 128 + r] = l;
-      ptx::tc_fence_before();
-      ptx::named_bar_sync(3, 256);
+      tg += n;
+      // Epilogue: wait for the item's last PV into O_g, normalise, and write the rows (bf16) out
+      // through shared memory: each warp stages the rows of lanes 0-15, then those of lanes 16-31,
+      // and its lane 0 issues one TMA store per half (rows past Nq are clipped by the TMA unit). A
+      // staging half is rewritten only after its previous store has read it. pv_done[g] completes
+      // once per item in which query tile g has a live tile.
+      wt.wait(BAR(pv_done[grp]), pv_phase & 1);
+      ++pv_phase;
       ptx::tc_fence_after();
-      const float mu0 = epi[0 * 128 + r], l0 = epi[1 * 128 + r];
-      const float mu1 = epi[2 * 128 + r], l1 = epi[3 * 128 + r];
-      // group g holds a partial iff it had a tile in this item (both do when n >= 2)
-      const bool has0 = ((0u - t0) & 1u) < uint32_t(it.n);
-      const bool has1 = ((1u - t0) & 1u) < uint32_t(it.n);
-      const float mm = has0 && has1 ? fmaxf(mu0, mu1) : (has0 ? mu0 : mu1);
-      const float a0 = has0 ? ptx::ex2(mu0 - mm) : 0.f;
-      const float a1 = has1 ? ptx::ex2(mu1 - mm) : 0.f;
-      const float lt = a0 * l0 + a1 * l1;
-      const float inv_l = 1.f / lt;
-      const float w0 = a0 * inv_l, w1 = a1 * inv_l;
-      // The group's D/2 columns of O, combined and rounded to bf16, leave through shared memory:
-      // each warp stages the rows of lanes 0-15, then those of lanes 16-31, and its lane 0 issues
-      // one TMA store per half (rows past Nq are clipped by the TMA unit). The threads never wait
-      // for global memory; a staging half is rewritten only after its previous store has read it.
-      uint32_t ow[D / 4];  // this row's D/2 bf16 columns, packed in pairs
+      const float inv_l = 1.f / l;
+      uint32_t ow[D / 2];  // the row's D columns, packed in bf16 pairs
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        const int col = grp * (D / 2) + c * 32;
-        uint32_t r0[32], r1[32];
-        ptx::tmem_ld32(tmem + lane_base + C::O_COL + 0 * D + col, r0);
-        ptx::tmem_ld32(tmem + lane_base + C::O_COL + 1 * D + col, r1);
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t rr[32];
+        ptx::tmem_ld32(tmem + lane_base + C::O_COL + grp * D + c * 32, rr);
         ptx::tmem_wait_ld();
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
-          // an accumulator without a partial may hold stale data: select, never multiply by zero
-          const float o0 = (has0 ? w0 * __uint_as_float(r0[2 * x]) : 0.f) +
-                           (has1 ? w1 * __uint_as_float(r1[2 * x]) : 0.f);
-          const float o1 = (has0 ? w0 * __uint_as_float(r0[2 * x + 1]) : 0.f) +
-                           (has1 ? w1 * __uint_as_float(r1[2 * x + 1]) : 0.f);
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(o0, o1);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(rr[2 * x]) * inv_l,
+                                                    __uint_as_float(rr[2 * x + 1]) * inv_l);
           ow[c * 16 + x] = *reinterpret_cast<uint32_t*>(&h2);
         }
       }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(BAR(o_free[grp]));
       {
-        uint8_t* stage = smem + C::OFF_OST + (grp * 4 + quarter) * C::OST_WARP;
         const int srow = lane & (C::OST_ROWS - 1);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -698,28 +708,24 @@ __global__ void __launch_bounds__(320, 1)
           __syncwarp();
           if ((lane >> 4) == half) {
 #pragma unroll
-            for (int x = 0; x < D / 16; ++x) {
-              // 16-byte chunk x of the row; 128-byte swizzle (chunk ^ row % 8) for D = 128
-              const int pc = D == 128 ? (x ^ (srow & 7)) : x;
-              *reinterpret_cast<uint4*>(stage + srow * D + pc * 16) =
-                  make_uint4(ow[4 * x], ow[4 * x + 1], ow[4 * x + 2], ow[4 * x + 3]);
+            for (int c = 0; c < D / 8; ++c) {
+              // 16-byte chunk c of the row: panel c/8, 128-byte swizzle (chunk ^ row % 8) inside it
+              const int x = c & 7;
+              *reinterpret_cast<uint4*>(stage + (c >> 3) * C::OST_PANEL + srow * 128 + ((x ^ (srow & 7)) << 4)) =
+                  make_uint4(ow[4 * c], ow[4 * c + 1], ow[4 * c + 2], ow[4 * c + 3]);
             }
           }
           ptx::fence_proxy_async_smem();
           __syncwarp();
           const int row_in_tile = quarter * 32 + half * C::OST_ROWS;
-          if (lane == 0 && row_in_tile < C::BQ && it.qi * C::BQ + row_in_tile < p.Nq) {
-            ptx::tma_store_5d(&tmO, ptx::smem_addr(stage), grp * (D / 2) % 64, it.qi * C::BQ + row_in_tile,
-                              grp * (D / 2) / 64, it.h, it.b);
+          if (lane == 0 && qi < p.Tq && row_in_tile < C::BQ && qi * C::BQ + row_in_tile < p.Nq) {
+            ptx::tma_store_5d(&tmO, ptx::smem_addr(stage), 0, qi * C::BQ + row_in_tile, 0, it.h, it.b);
             ptx::bulk_commit_group();
           }
         }
       }
-      if (valid_row && grp == 0 && p.lse)
-        p.lse[(size_t(it.b) * p.H + it.h) * p.Nq + n_row] = (mm + __log2f(lt)) * 0.6931471805599453f;
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(BAR(o_free));
-      t0 += it.n;
+      if (valid_row && p.lse)
+        p.lse[(size_t(it.b) * p.H + it.h) * p.Nq + n_row] = (m_used + __log2f(l)) * 0.6931471805599453f;
     }
     // the staged O rows must have been written out before the CTA (and its shared memory) ends
     if (lane == 0) ptx::bulk_wait_group0();

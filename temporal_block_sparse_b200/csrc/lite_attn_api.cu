@@ -134,20 +134,6 @@ bool make_tmap(CUtensorMap* map, const void* ptr, int B, int N, int H, int d, in
   return r == CUDA_SUCCESS;
 }
 
-// O as the epilogue stores it: the same 5-D view as q, a box of 16 rows of one softmax group's
-// d/2 columns (64 columns in one 128-byte swizzled panel for d = 128; 32 columns, unswizzled, for
-// d = 64).
-bool make_tmap_o(CUtensorMap* map, void* ptr, int B, int N, int H, int d) {
-  cuuint64_t dims[5] = {64, cuuint64_t(N), cuuint64_t(d / 64), cuuint64_t(H), cuuint64_t(B)};
-  cuuint64_t strides[4] = {cuuint64_t(H) * d * 2, 128, cuuint64_t(d) * 2, cuuint64_t(N) * H * d * 2};
-  cuuint32_t box[5] = {cuuint32_t(d / 2), 16, 1, 1, 1};
-  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, ptr, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                        CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 float resolve_scale(float scale, int d) {
   if (!(scale > 0.f) || std::isnan(scale)) return 1.0f / std::sqrt(static_cast<float>(d));
   return scale;
@@ -165,7 +151,7 @@ int launch_attention(DeviceCache* dc, int cfg_slot, const void* q, const void* k
   }
   CUtensorMap tq, tk, tv, to;
   if (!make_tmap(&tq, q, p.B, p.Nq, p.H, D, C::BQ) || !make_tmap(&tk, k, p.B, p.Nk, p.H, D, BN) ||
-      !make_tmap(&tv, v, p.B, p.Nk, p.H, D, BN) || !make_tmap_o(&to, p.o, p.B, p.Nq, p.H, D))
+      !make_tmap(&tv, v, p.B, p.Nk, p.H, D, BN) || !make_tmap(&to, p.o, p.B, p.Nq, p.H, D, C::OST_ROWS))
     return LITE_ERR_CUDA;
   int grid = dc->sms;
   if (g_opt.max_ctas > 0 && g_opt.max_ctas < grid) grid = g_opt.max_ctas;
@@ -198,7 +184,8 @@ lite::AttnParams base_params(void* o, float* lse, int B, int H, int Nq, int Nk, 
   p.Tq = (Nq + t - 1) / t;
   p.Tk = (Nk + t - 1) / t;
   p.W = (p.Tk + 31) / 32;
-  p.n_items = B * H * p.Tq;
+  p.Pq = (p.Tq + 1) / 2;
+  p.n_items = B * H * p.Pq;  // work items: pairs of query tiles
   p.scale_log2 = resolve_scale(scale, d) * 1.4426950408889634f;
   p.tau_log2 = -INFINITY;
   p.status = dc->status;
@@ -288,7 +275,7 @@ int range_bits(const int32_t* r, int n, int Nk, int t, bool whole, uint32_t* bit
 int enqueue_fwd(DeviceCache* dc, const FwdArgs& a, const lite::RangeBits* ranges, char* base, cudaStream_t s) {
   const FwdScratch f = fwd_scratch(a);
   lite::AttnParams p = base_params(a.o, a.lse, a.B, a.H, a.Nq, a.Nk, a.d, a.scale, dc);
-  const int Tq = p.Tq, Tk = p.Tk, W = p.W, rows = p.n_items;
+  const int Tq = p.Tq, Tk = p.Tk, W = p.W, rows = a.B * a.H * Tq;
   int16_t* list = reinterpret_cast<int16_t*>(base);
   int32_t* counts = reinterpret_cast<int32_t*>(base + f.list_b);
   int32_t* order = reinterpret_cast<int32_t*>(base + f.list_b + f.cnt_b);
@@ -304,14 +291,14 @@ int enqueue_fwd(DeviceCache* dc, const FwdArgs& a, const lite::RangeBits* ranges
                                                              lite::RangeBits{});
   if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
   if (g_opt.schedule) {
-    const size_t sm = size_t(a.B * a.H + Tq) * sizeof(int32_t);
-    lite::lite_schedule_kernel<<<a.B * a.H, 512, sm, s>>>(counts, order, a.B * a.H, Tq);
+    const size_t sm = size_t(a.B * a.H + p.Pq) * sizeof(int32_t);
+    lite::lite_schedule_kernel<2><<<a.B * a.H, 512, sm, s>>>(counts, order, a.B * a.H, Tq);
     if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
   }
   p.mask_out = a.mask_out;
   p.list = list;
   p.counts = counts;
-  p.order = g_opt.schedule ? order : nullptr;  // null: rows in their natural order
+  p.order = g_opt.schedule ? order : nullptr;  // null: pairs in their natural order
   p.work_counter = counter;
   p.tau_log2 = a.tau * 1.4426950408889634f;
   p.skip_test = (a.mask_out != nullptr && a.tau > -INFINITY) ? 1 : 0;
@@ -446,7 +433,7 @@ int lite_schedule(const int32_t* counts, int32_t* order, int B, int H, int T, li
   if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
   const int BH = B * H;
   const size_t sm = size_t(BH + T) * sizeof(int32_t);
-  lite::lite_schedule_kernel<<<BH, 512, sm, as_stream(stream)>>>(counts, order, BH, T);
+  lite::lite_schedule_kernel<1><<<BH, 512, sm, as_stream(stream)>>>(counts, order, BH, T);
   return cudaGetLastError() == cudaSuccess ? LITE_OK : LITE_ERR_CUDA;
 }
 

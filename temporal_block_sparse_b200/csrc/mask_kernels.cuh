@@ -8,8 +8,9 @@
 //    live set is (not masked or must-do) and not (must-skip and not must-do); must-do entries are
 //    tagged so that the attention kernel never flags them. The copied mask is mask_in unchanged.
 //  * lite_schedule_kernel: one CTA per head. Ranks the head among all heads by total live work,
-//    then places each of its query tiles by (live count desc, index asc) with an O(T^2) rank count
-//    in shared memory -- deterministic, no atomics on the output.
+//    then places each of its work items (query tiles, or pairs of query tiles) by (live count
+//    desc, index asc) with an O(T^2) rank count in shared memory -- deterministic, no atomics on
+//    the output.
 #pragma once
 
 #include <stdint.h>
@@ -137,9 +138,14 @@ __global__ void __launch_bounds__(256) lite_ranges_kernel(const uint32_t* __rest
 }
 
 // smem: totals[BH] ints, then counts of this head [T] ints
+// G = 1 orders the query tiles of every head; G = 2 orders pairs of consecutive query tiles
+// (2i, 2i+1), the work items of the attention kernel, by their combined live count. Output entries
+// are head * ceil(T/G) + item.
+template <int G>
 __global__ void __launch_bounds__(512) lite_schedule_kernel(const int32_t* __restrict__ counts,
                                                            int32_t* __restrict__ order, int BH, int T) {
   extern __shared__ int32_t sh[];
+  const int P = (T + G - 1) / G;  // items per head
   int32_t* totals = sh;
   int32_t* mine = sh + BH;
   const int g = blockIdx.x;
@@ -150,7 +156,13 @@ __global__ void __launch_bounds__(512) lite_schedule_kernel(const int32_t* __res
     const int v = __ldg(counts + x);
     if (v) atomicAdd(&totals[x / T], v);
   }
-  for (int x = threadIdx.x; x < T; x += blockDim.x) mine[x] = __ldg(counts + size_t(g) * T + x);
+  for (int x = threadIdx.x; x < P; x += blockDim.x) {
+    int c = 0;
+#pragma unroll
+    for (int k = 0; k < G; ++k)
+      if (G * x + k < T) c += __ldg(counts + size_t(g) * T + G * x + k);
+    mine[x] = c;
+  }
   __syncthreads();
   // rank of this head: heads with more work, or equal work and a lower index, go first
   const int my_total = totals[g];
@@ -162,15 +174,15 @@ __global__ void __launch_bounds__(512) lite_schedule_kernel(const int32_t* __res
     before += (totals[x] > my_total) || (totals[x] == my_total && x < g);
   atomicAdd(&rank_acc, before);
   __syncthreads();
-  const size_t base = size_t(rank_acc) * T;
-  for (int i = threadIdx.x; i < T; i += blockDim.x) {
+  const size_t base = size_t(rank_acc) * P;
+  for (int i = threadIdx.x; i < P; i += blockDim.x) {
     const int c = mine[i];
     int pos = 0;
-    for (int x = 0; x < T; ++x) {
+    for (int x = 0; x < P; ++x) {
       const int cx = mine[x];
       pos += (cx > c) || (cx == c && x < i);
     }
-    order[base + pos] = g * T + i;
+    order[base + pos] = g * P + i;
   }
 }
 
