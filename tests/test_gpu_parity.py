@@ -154,6 +154,37 @@ def test_optional_outputs_and_no_mask():
     assert_within(compare(o2, lse2, m, ref))
 
 
+@pytest.mark.parametrize("d,gw", [(64, 15), (128, 14)])
+def test_paired_query_tiles_with_disjoint_lists(d, gw):
+    """The kernel pairs query tiles (2i, 2i+1) and walks the union of their Skip-Lists. Here the
+    two tiles of each pair have disjoint live sets: even key tiles for one, odd for the other, so
+    every union tile is live for one query tile only. One pair has a fully skipped tile, and an
+    odd tile count leaves the last query tile without a partner. All rows against the oracle,
+    three steps with QK-Skip on."""
+    tile = 64 if d == 64 else 128
+    w = wl.small_workload(1, 2, 5, 9, gw, d, steps=3, locality=3.0, tau=-2.0, seed_offset=77 + d)
+    B, N, H = w.B, w.N, w.H
+    _, T, W = la.lite_mask_geometry(N, d)
+    assert T % 2 == 1 and N % tile != 0
+    bits = torch.zeros((B, H, T, W * 32), dtype=torch.bool)
+    for i in range(T):
+        bits[:, :, i, (i + 1) % 2:T:2] = True  # tile i skips the key tiles of the other parity
+    bits[:, 1, 2, :T] = True                   # head 1: query tile 2 fully skipped
+    weights = 2 ** torch.arange(32, dtype=torch.int64)
+    words = (bits.view(B, H, T, W, 32).to(torch.int64) * weights).sum(-1)
+    mask = torch.where(words >= 2 ** 31, words - 2 ** 32, words).to(torch.int32).cuda()
+    tr = wl.Trajectory(w, device="cuda")
+    for t in range(w.steps):
+        q, k, v = tr.current()
+        m_out = torch.empty_like(mask)
+        o, lse = la.lite_attn_fwd(q, k, v, mask, m_out, tau=-2.0)
+        assert la.lite_get_device_status() == 0
+        ref = oracle_step(q, k, v, mask, -2.0)
+        assert_within(compare(o, lse, m_out, ref))
+        mask = m_out
+        tr.advance()
+
+
 def test_fully_skipped_row_gives_zero_and_minus_inf():
     w = wl.small_workload(1, 1, 2, 8, 16, 128, seed_offset=4)  # N=256, T=2
     q, k, v = wl.Trajectory(w, device="cuda").current()
