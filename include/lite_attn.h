@@ -130,8 +130,9 @@ int lite_mask_to_ranges(const uint32_t* mask, int16_t* ranges, int32_t* nruns, i
                         int d, lite_stream_t stream);
 
 /*
- * lite_schedule -- work order for the persistent attention kernel (no counterpart on the pages;
- * it orders the query tiles that lite_attn_fwd processes).
+ * lite_schedule -- longest-first order of query tiles (no counterpart on the pages). The
+ * attention kernel behind lite_attn_fwd takes its work in pairs of consecutive query tiles (2i,
+ * 2i+1) of one head and orders those pairs the same way, by their combined live count.
  *
  * Heads (b, h) are ordered by decreasing total live-tile count (ties: lower b*H+h first); inside a
  * head, query tiles by decreasing live count (ties: lower index first). Writes order[B*H*T] with
@@ -167,9 +168,11 @@ const char* lite_status_string(int status);
  *  LITE_OPT_DEBUG_STALL    1 = test hook: the MMA warp of every CTA withholds its first tile, so
  *                          the waits that depend on it run out their limit (no fault, no hang).
  *  LITE_OPT_MAX_CTAS       cap on the persistent grid size (0 = one CTA per SM).
- *  LITE_OPT_SCHEDULE       1 (default) = lite_attn_fwd* hand out query tiles in the longest-first
- *                          order of lite_schedule; 0 = in their natural (b, h, tile) order, for
- *                          measuring what the schedule buys. Results are identical either way.
+ *  LITE_OPT_SCHEDULE       1 (default) = lite_attn_fwd* hand out their work items (pairs of
+ *                          consecutive query tiles of one head) longest first, heads kept
+ *                          together, as lite_schedule orders query tiles; 0 = in their natural
+ *                          (b, h, pair) order, for measuring what the schedule buys. Results are
+ *                          identical either way.
  * Returns LITE_ERR_INVALID_ARG for an unknown option or out-of-range value.
  */
 enum { LITE_OPT_WAIT_LIMIT_NS = 1, LITE_OPT_DEBUG_STALL = 2, LITE_OPT_MAX_CTAS = 3, LITE_OPT_SCHEDULE = 4 };
@@ -178,7 +181,8 @@ int lite_set_option(int option, long long value);
 /*
  * lite_set_cta_timing -- measurement hook for load balance. While set, every attention kernel
  * launch writes, for each CTA b < capacity, buf[3b] = its start time, buf[3b+1] = its end time
- * (both the GPU's global nanosecond timer) and buf[3b+2] = the number of live tiles it processed.
+ * (both the GPU's global nanosecond timer) and buf[3b+2] = the number of live (query tile, key tile)
+ * pairs it computed.
  * buf is caller-owned device memory of 3 * capacity uint64 values (8-byte aligned), or NULL with
  * capacity 0 to stop. Host state, like lite_set_kernel_events.
  */
