@@ -91,6 +91,10 @@ template <int D, int BN>
 struct AttnCfg {
   static constexpr int BM = 128;                 // MMA M = TMEM lanes = query rows of a tile slot
   static constexpr int BQ = BN;                  // valid query rows per query tile
+  // Rows of query tile g sit at TMEM lanes / smem rows [g*ROW1, g*ROW1 + BQ). With 64-row tiles
+  // (d = 64) the second tile takes the upper half, so the useful softmax warps of the two groups
+  // fall on different scheduler partitions.
+  static constexpr int ROW1 = BM - BQ;
   static constexpr int THREADS = 320;            // producer warp, MMA warp, 2 softmax warpgroups
   static constexpr int NCHUNK = D / 64;          // 128-byte swizzle atoms along d
   static constexpr int Q_CHUNK = BM * 128;       // bytes between d-chunks of a Q tile in smem
@@ -333,10 +337,11 @@ __global__ void __launch_bounds__(320, 1)
     ptx::prefetch_tmap(&tmO);
   }
   if constexpr (C::BQ < C::BM) {
-    // Q rows past the query tile are never loaded; keep them zero so their S rows stay finite.
+    // Q rows outside the query tile are never loaded; keep them zero so their S rows stay finite.
     for (int g = 0; g < 2; ++g)
       for (int c = 0; c < C::NCHUNK; ++c) {
-        uint4* z = reinterpret_cast<uint4*>(smem + C::OFF_Q + g * C::Q_BYTES + c * C::Q_CHUNK + C::BQ * 128);
+        const int zrow = g == 0 ? C::BQ : 0;  // the rows of slot g that hold no query row
+        uint4* z = reinterpret_cast<uint4*>(smem + C::OFF_Q + g * C::Q_BYTES + c * C::Q_CHUNK + zrow * 128);
         for (int x = threadIdx.x; x < (C::BM - C::BQ) * 128 / 16; x += blockDim.x) z[x] = make_uint4(0, 0, 0, 0);
       }
     ptx::fence_proxy_async_smem();
@@ -411,7 +416,8 @@ __global__ void __launch_bounds__(320, 1)
         ptx::mbar_arrive_expect_tx(BAR(q_full), (it.n[0] > 0 ? C::Q_TX : 0u) + (it.n[1] > 0 ? C::Q_TX : 0u));
         for (int g = 0; g < 2; ++g)
           if (it.n[g] > 0)
-            ptx::tma_load_5d(sQ + g * C::Q_BYTES, &tmQ, BAR(q_full), 0, (2 * it.qp + g) * C::BQ, 0, it.h, it.b);
+            ptx::tma_load_5d(sQ + g * C::Q_BYTES + g * C::ROW1 * 128, &tmQ, BAR(q_full), 0, (2 * it.qp + g) * C::BQ, 0,
+                             it.h, it.b);
         q_armed = true;
         q_par = qn & 1;
         // the union of the two descending lists, highest key tile first
@@ -548,6 +554,10 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
     const uint32_t gbar = 1 + grp;                  // named barrier of this warpgroup (128 threads)
     uint8_t* stage = smem + C::OFF_OST + (grp * 4 + quarter) * C::OST_WARP;
+    // a warp whose 32 lanes hold no row of its group's query tile (64-row tiles only) keeps the
+    // group's barrier sequence but does no TMEM, exponential or store work
+    const int wrow = quarter * 32 - grp * C::ROW1;
+    const bool idle_warp = C::ROW1 > 0 && (wrow < 0 || wrow >= C::BQ);
     uint32_t tg = 0, items = 0, pv_phase = 0;
     while (true) {
       const int slot = items & 1;
@@ -560,8 +570,9 @@ __global__ void __launch_bounds__(320, 1)
       const int qi = 2 * it.qp + grp;
       const int n = it.n[grp];
       const int row = it.row0 + grp;
-      const int n_row = qi * C::BQ + r;
-      const bool valid_row = qi < p.Tq && r < C::BQ && n_row < p.Nq;
+      const int rq = r - grp * C::ROW1;  // row inside the query tile
+      const int n_row = qi * C::BQ + rq;
+      const bool valid_row = qi < p.Tq && rq >= 0 && rq < C::BQ && n_row < p.Nq;
       const size_t o_off = (size_t(it.b) * p.Nq + n_row) * p.H + it.h;
       const bool any = it.n[0] + it.n[1] > 0;
       if (n == 0) {
@@ -589,6 +600,8 @@ __global__ void __launch_bounds__(320, 1)
         wt.wait(BAR(s_full[grp]), t & 1);
         __syncwarp();
         ptx::tc_fence_after();
+        float loc = -INFINITY;  // the tile's row max (log2 units)
+        if (!idle_warp) {
         const uint32_t s_tmem = tmem + lane_base + C::S_COL + grp * BN;
         // the whole S row is read once and stays in registers for the max and the exponentials
         uint32_t sr[BN];
@@ -615,7 +628,7 @@ __global__ void __launch_bounds__(320, 1)
           m2 = ptx::fmax3(m2, s[x + 4], s[x + 5]);
           m3 = ptx::fmax3(m3, s[x + 6], s[x + 7]);
         }
-        const float loc = ptx::fmax3(m0, m1, fmaxf(m2, m3)) * p.scale_log2;
+        loc = ptx::fmax3(m0, m1, fmaxf(m2, m3)) * p.scale_log2;
         // lazy rescale of the accumulator: move the reference only when the tile max exceeds it by
         // more than kRescaleLog2. The previous PV into O_g was issued before this tile's QK, so it
         // has completed now that S is ready; the rescaled O is stored before P is released.
@@ -659,11 +672,12 @@ __global__ void __launch_bounds__(320, 1)
           ptx::tmem_st16(s_tmem + c * 16, pk);
         }
         ptx::tmem_wait_st();
+        const float2 acc2 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+        l += acc2.x + acc2.y;
+        }
         ptx::tc_fence_before();
         ptx::mbar_arrive(BAR(p_full[grp]));
         if (r == 0) LITE_TRACE(2 + grp, 2, t);
-        const float2 acc2 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-        l += acc2.x + acc2.y;
         if (p.skip_test) {
           // QK-Skip, off the path from S to P: flag key tile j when loc - m < tau for every valid
           // row, m the running max over the tile's earlier live key tiles
@@ -687,7 +701,7 @@ __global__ void __launch_bounds__(320, 1)
       const float inv_l = 1.f / l;
       uint32_t ow[D / 2];  // the row's D columns, packed in bf16 pairs
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 32 && !idle_warp; ++c) {
         uint32_t rr[32];
         ptx::tmem_ld32(tmem + lane_base + C::O_COL + grp * D + c * 32, rr);
         ptx::tmem_wait_ld();
@@ -700,7 +714,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(BAR(o_free[grp]));
-      {
+      if (!idle_warp) {
         const int srow = lane & (C::OST_ROWS - 1);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -717,7 +731,7 @@ __global__ void __launch_bounds__(320, 1)
           }
           ptx::fence_proxy_async_smem();
           __syncwarp();
-          const int row_in_tile = quarter * 32 + half * C::OST_ROWS;
+          const int row_in_tile = wrow + half * C::OST_ROWS;
           if (lane == 0 && qi < p.Tq && row_in_tile < C::BQ && qi * C::BQ + row_in_tile < p.Nq) {
             ptx::tma_store_5d(&tmO, ptx::smem_addr(stage), 0, qi * C::BQ + row_in_tile, 0, it.h, it.b);
             ptx::bulk_commit_group();
