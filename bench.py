@@ -515,35 +515,56 @@ def run_steady(la, qkv, mask_in, tau, N, d, tile, T, dense_flop, warmup=5, reps=
             "attn_ms": attn / reps, "compact_ms": compact_ms, "schedule_ms": schedule_ms}
 
 
+def e2e_head_groups(B: int, H: int, T: int, sms: int, max_groups: int = 8) -> int:
+    """Head-group count for the end-to-end pipeline: the divisor g of H (g <= max_groups) with the
+    fewest rounds of pair items per step over the persistent grid (g calls of ceil(B*(H/g)*
+    ceil(T/2) / sms) rounds), the most groups among those (a shorter pipeline fill)."""
+    pairs = (T + 1) // 2
+    best, best_rounds = 1, None
+    for g in range(1, max_groups + 1):
+        if H % g:
+            continue
+        rounds = g * -(-(B * (H // g) * pairs) // sms)
+        if best_rounds is None or rounds <= best_rounds:
+            best, best_rounds = g, rounds
+    return best
+
+
 def run_e2e(args, la, wl, qkv, masks, dev, world, dist):
     """Same K steps through host buffers: H2D of q/k/v and D2H of o/lse inside the timed region.
 
-    Copies are double buffered, so step t+1's inputs upload while step t computes, and run on two
-    side streams, uploads on one and read-backs on the other: PCIe carries both directions at once,
-    so the read-back of step t overlaps the upload of step t+1.
+    Heads are independent, so each step runs as several calls of the public lite_attn_fwd on
+    consecutive head groups ([B, N, H/groups, d] each, with its own Skip-Mask rows), as a caller
+    streaming a layer through PCIe would (group count from e2e_head_groups). Group i+1 uploads while group i computes (two device
+    slots), on a copy stream; read-backs run on a third stream, so PCIe carries both directions at
+    once. The host holds each step's inputs per head group in pinned memory.
     """
     B, N, H, d = wl.B, wl.N, wl.H, wl.d
+    _, T, _ = la.lite_mask_geometry(N, d)
+    groups = e2e_head_groups(B, H, T, torch.cuda.get_device_properties(dev).multi_processor_count)
+    Hg = H // groups
     timed = list(range(args.warmup, args.warmup + args.steps))
-    host_in = []
+    units = [(t, g) for t in timed for g in range(groups)]
+    host_in = {}
     for t in timed:
-        bufs = tuple(torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in qkv[t])
-        for hb, x in zip(bufs, qkv[t]):
-            hb.copy_(x)
-        host_in.append(bufs)
-    host_o = [torch.empty((B, N, H, d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    host_l = [torch.empty((B, H, N), dtype=torch.float32).pin_memory() for _ in range(2)]
-    dev_in = [tuple(torch.empty_like(x) for x in qkv[0]) for _ in range(2)]
-    dev_o = [torch.empty((B, N, H, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
-    dev_l = [torch.empty((B, H, N), dtype=torch.float32, device=dev) for _ in range(2)]
-    e_masks = [m.clone() for m in masks]
+        for g in range(groups):
+            host_in[t, g] = tuple(x[:, :, g * Hg:(g + 1) * Hg].contiguous().cpu().pin_memory() for x in qkv[t])
+    host_o = [torch.empty((B, N, Hg, d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    host_l = [torch.empty((B, Hg, N), dtype=torch.float32).pin_memory() for _ in range(2)]
+    dev_in = [tuple(torch.empty((B, N, Hg, d), dtype=torch.bfloat16, device=dev) for _ in range(3)) for _ in range(2)]
+    dev_o = [torch.empty((B, N, Hg, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    dev_l = [torch.empty((B, Hg, N), dtype=torch.float32, device=dev) for _ in range(2)]
+    # each head group's Skip-Mask chain over the steps, starting from the same masks as the device run
+    g_masks = {(t, g): masks[t][:, g * Hg:(g + 1) * Hg].contiguous() for t in timed + [timed[-1] + 1]
+               for g in range(groups)}
     comp = torch.cuda.current_stream()
     copy = torch.cuda.Stream()   # host -> device
     back = torch.cuda.Stream()   # device -> host
     up_done = [torch.cuda.Event() for _ in range(2)]
     comp_done = [torch.cuda.Event() for _ in range(2)]
     down_done = [torch.cuda.Event() for _ in range(2)]
-    h2d = sum(x.numel() * x.element_size() for x in host_in[0])
-    d2h = host_o[0].numel() * 2 + host_l[0].numel() * 4
+    h2d = sum(x.numel() * x.element_size() for x in host_in[timed[0], 0]) * groups
+    d2h = (host_o[0].numel() * 2 + host_l[0].numel() * 4) * groups
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
         dist.barrier()
@@ -554,21 +575,22 @@ def run_e2e(args, la, wl, qkv, masks, dev, world, dist):
         s = i % 2
         with torch.cuda.stream(copy):
             if i >= 2:
-                copy.wait_event(comp_done[s])  # slot free once step i-2 has computed
-            for dst, src in zip(dev_in[s], host_in[i]):
+                copy.wait_event(comp_done[s])  # slot free once unit i-2 has computed
+            for dst, src in zip(dev_in[s], host_in[units[i]]):
                 dst.copy_(src, non_blocking=True)
             up_done[s].record(copy)
 
     upload(0)
-    for i, t in enumerate(timed):
+    for i, (t, g) in enumerate(units):
         s = i % 2
-        if i + 1 < len(timed):
+        if i + 1 < len(units):
             upload(i + 1)
         comp.wait_event(up_done[s])
         if i >= 2:
             comp.wait_event(down_done[s])  # output slot read back
         q, k, v = dev_in[s]
-        la.lite_attn_fwd(q, k, v, e_masks[t], e_masks[t + 1], tau=tau_at(wl, t, args.tau), o=dev_o[s], lse=dev_l[s])
+        la.lite_attn_fwd(q, k, v, g_masks[t, g], g_masks[t + 1, g], tau=tau_at(wl, t, args.tau), o=dev_o[s],
+                         lse=dev_l[s])
         comp_done[s].record(comp)
         with torch.cuda.stream(back):
             back.wait_event(comp_done[s])
@@ -582,8 +604,9 @@ def run_e2e(args, la, wl, qkv, masks, dev, world, dist):
     ms = max_over_ranks(start.elapsed_time(end), dist, dev)
     value = wl.dense_flop() * len(timed) * world / (ms * 1e-3) / 1e12
     return {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "ms_per_step": ms / len(timed),
-            "note": "pinned host q/k/v in, o/lse out; uploads and read-backs on two streams, overlapping compute"}
+            "ms_per_step": ms / len(timed), "head_groups": groups,
+            "note": f"pinned host q/k/v in, o/lse out; each step as {groups} lite_attn_fwd calls on consecutive "
+                    "head groups, uploads of the next group and read-backs on two streams overlapping compute"}
 
 
 # --------------------------------------------------------------------------------- studies

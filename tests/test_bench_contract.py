@@ -34,3 +34,20 @@ def test_reference_arm_json_line():
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_e2e_head_groups():
+    """The end-to-end pipeline's head-group count: a divisor of H, fewest rounds of pair items
+    over the persistent grid per step, then the most groups."""
+    import bench
+
+    # 480p: 40 heads x 128 pairs over 148 CTAs. One call takes 35 rounds, 4 groups 4 x 9 = 36,
+    # 5 groups 5 x 7 = 35: five groups of eight heads.
+    assert bench.e2e_head_groups(1, 40, 256, 148) == 5
+    # 720p: 296 pairs a head; 8 groups of five heads take 8 x 10 = 80 rounds, as one call does
+    assert bench.e2e_head_groups(1, 40, 591, 148) == 8
+    # few items: never split a call that fits in one round
+    assert bench.e2e_head_groups(1, 1, 16, 148) == 1
+    assert bench.e2e_head_groups(1, 8, 256, 148) == 1
+    for H in (1, 3, 7, 12, 40):
+        assert H % bench.e2e_head_groups(1, H, 100, 148) == 0
