@@ -196,6 +196,15 @@ int lite_set_cta_timing(void* buf, int capacity);
 int lite_set_kernel_events(void* before, void* after);
 
 /*
+ * lite_scratch_pool_bytes -- measurement hook. *reserved = device memory, in bytes, that the
+ * library's scratch pool on the current device holds (its stream-ordered pool keeps freed memory
+ * for reuse); 0 while no pooled call has run on the device, since the pool is created by the
+ * first lite_attn_fwd / lite_attn_fwd_ex call. Makes no allocation. LITE_ERR_INVALID_ARG for a
+ * NULL pointer.
+ */
+int lite_scratch_pool_bytes(long long* reserved);
+
+/*
  * lite_attn_fwd_noalloc -- lite_attn_fwd for callers that must not allocate device memory.
  *
  * The LiteAttention paper and pages have no counterpart to this entry point; it exists for
@@ -208,7 +217,9 @@ int lite_set_kernel_events(void* before, void* after);
  * where the per-call scratch (live lists, counts, work order, work counter) lives: in one fixed
  * array of LITE_NOALLOC_SCRATCH_BYTES (8 MiB) that the library defines in device memory. Every GPU
  * that loads the library holds that array until the process exits. This call makes no cudaMalloc,
- * cudaFree or other allocating call.
+ * cudaFree or other allocating call, and creates no memory pool (the scratch pool behind
+ * lite_attn_fwd is created by the first lite_attn_fwd / lite_attn_fwd_ex call on a device, never
+ * by this one; lite_scratch_pool_bytes reports whether it exists).
  *
  *  - Limit: the layer's scratch must fit in 8 MiB. With R = B*H*T and T = ceil(N / tile) it is
  *    up256(2*R*T) + 2*up256(4*R) + 256 bytes (up256 rounds up to a multiple of 256), about
@@ -216,7 +227,8 @@ int lite_set_kernel_events(void* before, void* after);
  *    (N=75600: 28 MB) does not. Layers that do not fit return LITE_ERR_SCRATCH_LIMIT before any
  *    work is enqueued.
  *  - Set-up: the first call on each device looks up the array's device address (with that device
- *    current); make that first call before capturing any stream into a CUDA graph.
+ *    current), the device's SM count and the status word's address; make that first call before
+ *    capturing any stream into a CUDA graph.
  *  - Sharing: all calls on a device use the same array, and it keeps whatever the last call left
  *    in it (the work counter is cleared on the stream at the start of every call). Calls whose
  *    work overlaps on the GPU -- for example on two streams without ordering between them --

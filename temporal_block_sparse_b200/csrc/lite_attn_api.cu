@@ -44,6 +44,7 @@ long long* g_trace = nullptr;
 
 struct DeviceCache {
   bool init = false;
+  int dev = 0;
   int sms = 0;
   int* status = nullptr;
   bool smem_set[4] = {false, false, false, false};
@@ -59,6 +60,9 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 cudaStream_t as_stream(lite_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// Per-device set-up that every entry point needs: SM count, the status word's device address and
+// the tensor-map encoder. It allocates nothing; the scratch pool is created separately, on the first
+// pooled call (ensure_pool).
 int device_cache(DeviceCache** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LITE_ERR_CUDA;
@@ -68,14 +72,7 @@ int device_cache(DeviceCache** out) {
     if (cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return LITE_ERR_CUDA;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&c.status), g_device_status) != cudaSuccess)
       return LITE_ERR_CUDA;
-    cudaMemPoolProps props;
-    std::memset(&props, 0, sizeof(props));
-    props.allocType = cudaMemAllocationTypePinned;
-    props.location.type = cudaMemLocationTypeDevice;
-    props.location.id = dev;
-    if (cudaMemPoolCreate(&c.pool, &props) != cudaSuccess) return LITE_ERR_CUDA;
-    uint64_t keep = ~uint64_t(0);
-    if (cudaMemPoolSetAttribute(c.pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) return LITE_ERR_CUDA;
+    c.dev = dev;
     c.init = true;
   }
   if (!g_encode) {
@@ -87,6 +84,26 @@ int device_cache(DeviceCache** out) {
     g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
   *out = &c;
+  return LITE_OK;
+}
+
+// The library-owned stream-ordered pool of a device, created on first use by a pooled call.
+int ensure_pool(DeviceCache* c) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (c->pool) return LITE_OK;
+  cudaMemPoolProps props;
+  std::memset(&props, 0, sizeof(props));
+  props.allocType = cudaMemAllocationTypePinned;
+  props.location.type = cudaMemLocationTypeDevice;
+  props.location.id = c->dev;
+  cudaMemPool_t pool = nullptr;
+  if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return LITE_ERR_CUDA;
+  uint64_t keep = ~uint64_t(0);
+  if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
+    cudaMemPoolDestroy(pool);
+    return LITE_ERR_CUDA;
+  }
+  c->pool = pool;
   return LITE_OK;
 }
 
@@ -308,7 +325,7 @@ int enqueue_fwd(DeviceCache* dc, const FwdArgs& a, const lite::RangeBits* ranges
 // pool-backed scratch around enqueue_fwd
 int fwd_pooled(const FwdArgs& a, const lite::RangeBits* ranges, cudaStream_t s) {
   DeviceCache* dc = nullptr;
-  if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
+  if (device_cache(&dc) != LITE_OK || ensure_pool(dc) != LITE_OK) return LITE_ERR_CUDA;
   const FwdScratch f = fwd_scratch(a);
   void* ws = nullptr;
   if (cudaMallocFromPoolAsync(&ws, f.total, dc->pool, s) != cudaSuccess) return LITE_ERR_CUDA;
@@ -380,6 +397,18 @@ int lite_set_kernel_events(void* before, void* after) {
   if ((before == nullptr) != (after == nullptr)) return LITE_ERR_INVALID_ARG;
   g_ev_before = static_cast<cudaEvent_t>(before);
   g_ev_after = static_cast<cudaEvent_t>(after);
+  return LITE_OK;
+}
+
+int lite_scratch_pool_bytes(long long* reserved) {
+  if (!reserved) return LITE_ERR_INVALID_ARG;
+  DeviceCache* dc = nullptr;
+  if (device_cache(&dc) != LITE_OK) return LITE_ERR_CUDA;
+  *reserved = 0;
+  if (!dc->pool) return LITE_OK;
+  cuuint64_t v = 0;
+  if (cudaMemPoolGetAttribute(dc->pool, cudaMemPoolAttrReservedMemCurrent, &v) != cudaSuccess) return LITE_ERR_CUDA;
+  *reserved = static_cast<long long>(v);
   return LITE_OK;
 }
 

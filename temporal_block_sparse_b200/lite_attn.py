@@ -51,6 +51,7 @@ SIGNATURES = {
     "lite_dropped_mass": ([_P, _P, _P, _P, _I, _I, _I, _P], _I),
     "lite_mask_to_ranges": ([_P, _P, _P, _I, _I, _I, _I, _P], _I),
     "lite_set_cta_timing": ([_P, _I], _I),
+    "lite_scratch_pool_bytes": ([ctypes.POINTER(ctypes.c_longlong)], _I),
 }
 MAX_MERGE_PARTS = 8
 
@@ -115,6 +116,8 @@ def _check_qkv(q, k, v):
         _check_bf16(name, t)
     if not (q.shape == k.shape == v.shape):
         raise ValueError("q, k, v must have the same shape [B, N, H, d]")
+    if not (q.device == k.device == v.device):
+        raise ValueError("q, k, v must be on one device")
 
 
 def _check_qkv_cross(q, k, v):
@@ -122,6 +125,8 @@ def _check_qkv_cross(q, k, v):
         _check_bf16(name, t)
     if k.shape != v.shape or q.shape[0] != k.shape[0] or q.shape[2:] != k.shape[2:]:
         raise ValueError("q [B, Nq, H, d] and k, v [B, Nk, H, d] must agree in B, H and d")
+    if not (q.device == k.device == v.device):
+        raise ValueError("q, k, v must be on one device")
 
 
 def _ranges(r, name):
@@ -150,7 +155,7 @@ def lite_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask_in: Op
         o = torch.empty_like(q)
     if lse is None and return_lse:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    _check_masks(mask_in, mask_out)
+    _check_fwd_buffers(q, k, o, lse, mask_in, mask_out)
     st = load().lite_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _ptr(lse), _ptr(mask_in),
                               _ptr(mask_out), B, H, N, d, float(scale or 0.0), float(tau), _stream_handle(stream))
     _check("lite_attn_fwd", st)
@@ -167,6 +172,7 @@ def lite_attn_dense(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Op
         o = torch.empty_like(q)
     if lse is None and return_lse:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _check_outputs(q, o, lse)
     st = load().lite_attn_dense(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _ptr(lse), B, H, N, d,
                                 float(scale or 0.0), _stream_handle(stream))
     _check("lite_attn_dense", st)
@@ -226,6 +232,7 @@ def lite_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: 
     """
     _check_qkv(q, k, v)
     B, N, H, d = q.shape
+    _check_fwd_buffers(q, k, o, lse, mask_in, mask_out)
     st = load().lite_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _ptr(lse),
                                       _ptr(mask_in), _ptr(mask_out), B, H, N, d, float(scale or 0.0), float(tau),
                                       _stream_handle(stream))
@@ -233,10 +240,46 @@ def lite_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: 
     return o, lse
 
 
-def _check_masks(*masks):
+def _check_masks(*masks, shape=None, device=None):
+    """Skip-Masks: contiguous int32 CUDA tensors, of `shape` [B, H, Tq, Wk] and on `device` when given."""
     for m in masks:
-        if m is not None and (m.dtype != torch.int32 or not m.is_contiguous() or not m.is_cuda):
+        if m is None:
+            continue
+        if m.dtype != torch.int32 or not m.is_contiguous() or not m.is_cuda:
             raise ValueError("masks must be contiguous int32 CUDA tensors [B, H, Tq, Wk]")
+        if shape is not None and tuple(m.shape) != tuple(shape):
+            raise ValueError(f"mask shape {tuple(m.shape)} != [B, H, Tq, Wk] = {tuple(shape)}")
+        if device is not None and m.device != device:
+            raise ValueError("masks must be on the device of q")
+
+
+def _check_outputs(q: torch.Tensor, o: torch.Tensor, lse: Optional[torch.Tensor]):
+    """o: contiguous bf16 shaped like q [B, Nq, H, d]; lse: contiguous fp32 [B, H, Nq]; both on q's device."""
+    _check_bf16("o", o)
+    if o.shape != q.shape or o.device != q.device:
+        raise ValueError("o must have q's shape [B, Nq, H, d] and device")
+    if lse is not None:
+        B, Nq, H, _ = q.shape
+        if (lse.dtype != torch.float32 or not lse.is_contiguous() or not lse.is_cuda or lse.device != q.device
+                or tuple(lse.shape) != (B, H, Nq)):
+            raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, H, Nq] on q's device")
+
+
+def _check_fwd_buffers(q, k, o, lse, mask_in, mask_out):
+    """Every device buffer of a masked forward call, checked before the C call (the library cannot
+    tell a host pointer or a short buffer from a good one)."""
+    B, Nq, H, d = q.shape
+    _, Tq, _ = lite_mask_geometry(Nq, d)
+    _, _, Wk = lite_mask_geometry(k.shape[1], d)
+    _check_outputs(q, o, lse)
+    _check_masks(mask_in, mask_out, shape=(B, H, Tq, Wk), device=q.device)
+
+
+def scratch_pool_bytes() -> int:
+    """Device memory held by the library's scratch pool on the current device (0 before any pooled call)."""
+    v = ctypes.c_longlong(0)
+    _check("lite_scratch_pool_bytes", load().lite_scratch_pool_bytes(ctypes.byref(v)))
+    return int(v.value)
 
 
 def lite_attn_fwd_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask_in: Optional[torch.Tensor] = None,
@@ -252,7 +295,7 @@ def lite_attn_fwd_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask_in:
         o = torch.empty_like(q)
     if lse is None and return_lse:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
-    _check_masks(mask_in, mask_out)
+    _check_fwd_buffers(q, k, o, lse, mask_in, mask_out)
     do_arr, n_do = _ranges(must_do, "must_do")
     skip_arr, n_skip = _ranges(must_skip, "must_skip")
     st = load().lite_attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _ptr(lse), _ptr(mask_in),
@@ -274,6 +317,7 @@ def lite_attn_dense_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale:
         o = torch.empty_like(q)
     if lse is None and return_lse:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _check_outputs(q, o, lse)
     st = load().lite_attn_dense_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _ptr(lse), B, H, Nq, Nk,
                                    d, float(scale or 0.0), _stream_handle(stream))
     _check("lite_attn_dense_ex", st)

@@ -51,6 +51,10 @@ def test_geometry():
     assert lib.lite_mask_geometry(0, 64, None, None, None) == la.LITE_ERR_INVALID_ARG
 
 
+def test_scratch_pool_hook_refuses_null():
+    assert la.load().lite_scratch_pool_bytes(None) == la.LITE_ERR_INVALID_ARG
+
+
 def test_status_strings():
     for code in (0, -1, -2, -3, -4, -5, 7):
         s = la.status_string(code)

@@ -1,8 +1,9 @@
 """bench.py's reference arm (the oracle timed on the host cores) prints the contract's JSON line (CPU).
 
-The GPU arm needs a B200 and is exercised by the full test run; this checks, without a GPU, that the
-reference arm runs on a bounded sample and reports the same metric, unit and direction with the
-fields the contract names.
+The GPU arm needs a B200; this checks, without a GPU, that the reference arm runs on a bounded
+sample of the default workload and reports the same metric, unit, direction and config with the
+fields the contract names, and the host-side rules of both arms (the trajectory bound, the
+end-to-end step count and head groups).
 """
 
 import json
@@ -27,8 +28,9 @@ def test_reference_arm_json_line():
     assert d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
     assert d["value"] > 0 and d["ms_per_step"] > 0
     assert d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 0
-    assert d["scaling"] == "weak" and d["data"] == "synthetic" and d["vs_baseline"] is None
-    assert d["config"]["workload"].startswith("480p")
+    assert d["scaling"] == "strong" and d["data"] == "synthetic" and d["vs_baseline"] is None
+    assert d["config"]["workload"].startswith("stress layer: B=2 H=40 N=75600")
+    assert d["config"]["B"] == 2 and d["config"]["H"] == 40 and d["config"]["tau"] == [-3.0]
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
     e2e = d["e2e"]
@@ -51,3 +53,46 @@ def test_e2e_head_groups():
     assert bench.e2e_head_groups(1, 8, 256, 148) == 1
     for H in (1, 3, 7, 12, 40):
         assert H % bench.e2e_head_groups(1, H, 100, 148) == 0
+
+
+def test_runs_stay_inside_the_trajectory():
+    """The default run (5 warm-up + 20 timed steps) fits the stress layer's 30 steps; a longer one
+    is refused rather than extended with a made-up threshold."""
+    import pytest
+
+    import bench
+    from temporal_block_sparse_b200 import workload as wl
+
+    w = wl.WORKLOADS[bench.DEFAULT_WORKLOAD]
+    assert w.steps == 30
+    bench.check_trajectory(w, 25)
+    bench.check_trajectory(w, 30)
+    with pytest.raises(SystemExit):
+        bench.check_trajectory(w, 31)
+    assert bench.tau_at(w, 29, None) == -3.0
+    with pytest.raises(ValueError):
+        bench.tau_at(w, 30, None)
+    with pytest.raises(ValueError):
+        bench.tau_at(wl.WORKLOADS["480p"], 10, None)
+
+
+def test_e2e_step_count():
+    import bench
+
+    gb = 1 << 30
+    assert bench.e2e_step_count(None, 20, 5 * gb, 600 * gb) == 20   # all fit in a third of the memory
+    assert bench.e2e_step_count(None, 20, 5 * gb, 60 * gb) == 4     # 20 GB for inputs -> 4 steps
+    assert bench.e2e_step_count(None, 20, 5 * gb, 1 * gb) == 1      # never fewer than one
+    assert bench.e2e_step_count(3, 20, 5 * gb, 1 * gb) == 3         # an explicit request wins
+    assert bench.e2e_step_count(50, 20, 5 * gb, 1 * gb) == 20       # ... up to the timed steps
+
+
+def test_mask_kernel_bytes():
+    import torch
+
+    import bench
+
+    m = torch.zeros((2, 40, 591, 19), dtype=torch.int32)
+    rows = 2 * 40 * 591
+    assert bench.mask_bytes(m, 1000, 591, with_copy=False) == rows * 19 * 4 + 2000 + rows * 4
+    assert bench.mask_bytes(m, 1000, 591, with_copy=True) == 2 * rows * 19 * 4 + 2000 + rows * 4

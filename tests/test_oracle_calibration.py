@@ -33,9 +33,10 @@ def _qkv(seed=0, H=2, frames=6, gh=8, gw=16, d=64, locality=5.0, tau=-2.0, steps
     return w, out
 
 
-def test_error_budget_schedule_shape():
+def _budget_pins(schedule):
+    """The schedule's stated shape and values derived by hand from it, for a schedule function."""
     for T, ratio in ((10, 0.3), (50, 0.3), (7, 0.5), (20, 0.0), (1, 0.3)):
-        b = cal.error_budgets(T, ratio)
+        b = np.asarray(schedule(T, ratio))
         n_early = int(T * ratio)
         assert len(b) == T
         assert np.all(np.diff(b) >= 0)                     # later steps never get a tighter budget
@@ -46,14 +47,66 @@ def test_error_budget_schedule_shape():
             steps = np.diff(b[:n_early])
             assert np.allclose(steps, steps[0] if len(steps) else 0)  # linear
     # hand-derived: 10 steps, 3 early steps rising by 1/6 each
-    assert np.allclose(cal.error_budgets(10), [0.5, 2 / 3, 5 / 6, 1, 1, 1, 1, 1, 1, 1])
+    assert np.allclose(schedule(10, 0.3), [0.5, 2 / 3, 5 / 6, 1, 1, 1, 1, 1, 1, 1])
 
 
-def test_tau_for_budget_scales_the_element_bound():
-    for base in (-10.0, -3.0, 0.0):
-        assert cal.tau_for_budget(base, 1.0) == base
-        for b in (0.5, 0.75):
-            assert math.isclose(math.exp(cal.tau_for_budget(base, b)), b * math.exp(base), rel_tol=1e-12)
+def test_error_budget_schedule_shape():
+    _budget_pins(cal.error_budgets)
+
+
+@pytest.mark.parametrize("mistake", ["reversed ramp", "ramp from zero", "ramp over every step"])
+def test_planted_mistake_in_budget_schedule_is_caught(monkeypatch, mistake):
+    """A mistake planted in oracle.calibration.error_budgets itself fails the pins above."""
+    right = cal.error_budgets
+
+    def planted(num_steps, early_step_ratio=0.3):
+        b = np.asarray(right(num_steps, early_step_ratio))
+        if mistake == "reversed ramp":         # early steps get MORE tolerance
+            return 1.5 - b
+        if mistake == "ramp from zero":        # the 0.5 offset dropped
+            return np.where(b < 1.0, 2 * b - 1.0, b)
+        return np.asarray(right(num_steps, 1.0))  # early_step_ratio ignored
+
+    monkeypatch.setattr(cal, "error_budgets", planted)
+    with pytest.raises(AssertionError):
+        _budget_pins(cal.error_budgets)
+
+
+def _flagged_tile_max_p(q, k, mask_out):
+    """Largest dense-softmax probability inside each flagged tile (numpy, float64, per head)."""
+    B, N, H, d = q.shape
+    t, T, _ = oracle.geometry(N, d)
+    out = []
+    for b in range(B):
+        for h in range(H):
+            s = (q[b, :, h] @ k[b, :, h].T) / math.sqrt(d)
+            p = np.exp(s - s.max(axis=1, keepdims=True))
+            p /= p.sum(axis=1, keepdims=True)
+            for i in range(T):
+                for j in range(T):
+                    if oracle.is_skipped(mask_out, b, h, i, j):
+                        out.append(p[i * t:(i + 1) * t, j * t:(j + 1) * t].max())
+    return np.asarray(out)
+
+
+def test_tau_for_budget_bounds_the_flagged_elements():
+    """tau_for_budget(base, b) is the threshold whose flags keep every element of a flagged tile
+    below b * exp(base) under that step's dense softmax (pinned through the forward pass's flags and
+    an independent softmax, not through the function's formula). A sign-flipped mapping flags
+    tiles that break the bound on the same inputs."""
+    _, steps = _qkv(seed=17, locality=5.0, H=2)
+    q, k, v = steps[0]
+    checked, caught = 0, 0
+    for base, b in ((-3.0, 0.05), (-2.0, 0.1), (-1.0, 0.5)):
+        tau = cal.tau_for_budget(base, b)
+        r = oracle.lite_attention_forward(q, k, v, None, tau=tau)
+        mx = _flagged_tile_max_p(q, k, r.mask_out)
+        checked += len(mx)
+        assert np.all(mx < b * math.exp(base))
+        wrong = oracle.lite_attention_forward(q, k, v, None, tau=base - math.log(b))
+        caught += int(np.any(_flagged_tile_max_p(q, k, wrong.mask_out) >= b * math.exp(base)))
+    assert checked > 0 and caught > 0
+    assert cal.tau_for_budget(-3.0, 1.0) == -3.0
 
 
 def test_dropped_mass_two_routes_agree():
@@ -129,12 +182,6 @@ def test_calibrate_step_keeps_mask_when_nothing_fits():
     assert r.tau == -np.inf
     np.testing.assert_array_equal(r.mask_out, m)
     assert math.isclose(r.dropped_max, base, rel_tol=1e-12)
-
-
-def test_planted_mistake_in_budget_direction_is_caught():
-    # a schedule that gives early steps MORE tolerance contradicts the pages and fails the shape pin
-    bad = 1.5 - np.asarray(cal.error_budgets(10))
-    assert not np.all(np.diff(bad) >= 0)
 
 
 def test_mean_criterion_is_looser_than_max():
