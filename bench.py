@@ -63,8 +63,8 @@ def parse_args():
     ap.add_argument("--study-steps", type=int, default=None)
     ap.add_argument("--eps", type=float, default=1e-2, help="base error budget of the calibration study")
     ap.add_argument("--e2e-steps", type=int, default=None,
-                    help="timed steps repeated end to end through host buffers (default: as many as fit in "
-                         "a third of the free host memory, at most all of them)")
+                    help="timed steps repeated end to end through host buffers (default: 5, fewer if their "
+                         "pinned inputs would not fit in a third of the free host memory)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     return ap.parse_args()
@@ -612,12 +612,17 @@ def e2e_head_groups(B: int, H: int, T: int, sms: int, max_groups: int = 8) -> in
     return best
 
 
+E2E_DEFAULT_STEPS = 5
+
+
 def e2e_step_count(requested, timed_steps: int, bytes_per_step: int, host_free: int) -> int:
-    """How many timed steps the end-to-end run repeats: the requested count, else as many as fit in
-    a third of the free host memory (pinned inputs of every repeated step), at least 1, at most all."""
+    """How many timed steps the end-to-end run repeats: the requested count, else E2E_DEFAULT_STEPS
+    or as many as fit in a third of the free host memory (the pinned inputs of every repeated
+    step), whichever is fewer; at least 1, at most all timed steps."""
     if requested:
         return max(1, min(int(requested), timed_steps))
-    return max(1, min(timed_steps, (host_free // 3) // max(bytes_per_step, 1)))
+    fit = (host_free // 3) // max(bytes_per_step, 1)
+    return max(1, min(timed_steps, E2E_DEFAULT_STEPS, fit))
 
 
 def run_e2e(args, la, wl, qkv, masks, dev, world, dist, H, attn_ms, elapsed_ms):

@@ -47,7 +47,7 @@ enum {
   LITE_ERR_UNSUPPORTED = -2, /* d not in {64, 128}, misaligned pointer, T or sizes beyond limits  */
   LITE_ERR_CUDA = -3,        /* a CUDA launch, allocation or query failed                          */
   LITE_ERR_TIMEOUT = -4,     /* device status: a kernel wait exceeded its time limit and gave up   */
-  LITE_ERR_CHECK = -5,       /* device status: an in-kernel consistency check failed               */
+  LITE_ERR_CHECK = -5,       /* device status: a kernel found a malformed Skip-List or work order  */
   LITE_ERR_SCRATCH_LIMIT = -6 /* lite_attn_fwd_noalloc: the layer needs more than its fixed scratch  */
 };
 
@@ -238,6 +238,35 @@ int lite_scratch_pool_bytes(long long* reserved);
 int lite_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                           const uint32_t* mask_in, uint32_t* mask_out, int B, int H, int N, int d,
                           float scale, float tau, lite_stream_t stream);
+
+/*
+ * lite_attn_fwd_list -- lite_attn_fwd over caller-supplied Skip-Lists instead of a Skip-Mask.
+ *
+ * The skill page "Lite Attention Temporal Sparse" (Architecture Overview) keeps the skip state as a
+ * bitmask "or Skip-List for high sparsity": per (b, h, query tile) the live key tiles, which the
+ * kernel visits from the highest index down (README, must_do_list: "we iterate in reverse order
+ * inside of the kernel"). lite_attn_fwd builds these lists from the mask (lite_mask_to_list) on every
+ * call; a caller that keeps the lists itself passes them here, and the compaction step and the mask
+ * copy are skipped. Results are those of lite_attn_fwd on the mask the lists describe.
+ *
+ *  list      in   device int16 [B, H, T, T]: row (b, h, i) holds counts[b, h, i] key-tile indices,
+ *                 strictly descending, each < T; bit 14 (0x4000) may tag an entry that must never
+ *                 be flagged (a must-do tile). Entries past the count are not read.
+ *  counts    in   device int32 [B, H, T], each in [0, T].
+ *  mask_out  in/out device uint32 [B, H, T, W], or NULL = do not record flags. Flags are OR-ed into
+ *                 it as they are found; nothing is copied into it first (initialise it, e.g. with
+ *                 the mask the lists came from).
+ *  Other arguments as lite_attn_fwd. Scratch (work order, counter: about 4*B*H*T bytes) comes from
+ *  the library's stream-ordered pool, as for lite_attn_fwd.
+ *
+ * The attention kernel checks every list it walks: a count outside [0, T], an entry with bits other
+ * than the index and the tag, an index >= T or one not below its predecessor stops the kernel
+ * before that tile is loaded, and lite_get_device_status then returns LITE_ERR_CHECK (the outputs
+ * of that call are invalid; the context stays usable).
+ */
+int lite_attn_fwd_list(const void* q, const void* k, const void* v, void* o, float* lse, const int16_t* list,
+                       const int32_t* counts, uint32_t* mask_out, int B, int H, int N, int d, float scale, float tau,
+                       lite_stream_t stream);
 
 /*
  * lite_attn_fwd_ex -- lite_attn_fwd for partial attention: queries and keys of different lengths,

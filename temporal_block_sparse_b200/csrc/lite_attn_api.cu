@@ -322,6 +322,36 @@ int enqueue_fwd(DeviceCache* dc, const FwdArgs& a, const lite::RangeBits* ranges
   return run_attention(dc, a.d, a.q, a.k, a.v, p, s);
 }
 
+// Schedule and attention over caller-supplied Skip-Lists (no compaction, no mask copy). Scratch:
+// work order [rows] int32 | work counter.
+size_t list_scratch_bytes(const FwdArgs& a) {
+  const int t = tile_for(a.d);
+  const size_t rows = size_t(a.B) * a.H * ((a.Nq + t - 1) / t);
+  return align256(rows * sizeof(int32_t)) + 256;
+}
+
+int enqueue_list(DeviceCache* dc, const FwdArgs& a, const int16_t* list, const int32_t* counts, char* base,
+                 cudaStream_t s) {
+  lite::AttnParams p = base_params(a.o, a.lse, a.B, a.H, a.Nq, a.Nk, a.d, a.scale, dc);
+  const int Tq = p.Tq, rows = a.B * a.H * Tq;
+  int32_t* order = reinterpret_cast<int32_t*>(base);
+  int32_t* counter = reinterpret_cast<int32_t*>(base + align256(size_t(rows) * sizeof(int32_t)));
+  if (cudaMemsetAsync(counter, 0, sizeof(int32_t), s) != cudaSuccess) return LITE_ERR_CUDA;
+  if (g_opt.schedule) {
+    const size_t sm = size_t(a.B * a.H + p.Pq) * sizeof(int32_t);
+    lite::lite_schedule_kernel<2><<<a.B * a.H, 512, sm, s>>>(counts, order, a.B * a.H, Tq);
+    if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
+  }
+  p.mask_out = a.mask_out;
+  p.list = list;
+  p.counts = counts;
+  p.order = g_opt.schedule ? order : nullptr;
+  p.work_counter = counter;
+  p.tau_log2 = a.tau * 1.4426950408889634f;
+  p.skip_test = (a.mask_out != nullptr && a.tau > -INFINITY) ? 1 : 0;
+  return run_attention(dc, a.d, a.q, a.k, a.v, p, s);
+}
+
 // pool-backed scratch around enqueue_fwd
 int fwd_pooled(const FwdArgs& a, const lite::RangeBits* ranges, cudaStream_t s) {
   DeviceCache* dc = nullptr;
@@ -356,7 +386,7 @@ const char* lite_status_string(int status) {
     case LITE_ERR_UNSUPPORTED: return "unsupported shape, head dim or alignment";
     case LITE_ERR_CUDA: return "CUDA launch, allocation or query failed";
     case LITE_ERR_TIMEOUT: return "a kernel wait exceeded its time limit; outputs of that call are invalid";
-    case LITE_ERR_CHECK: return "an in-kernel consistency check failed";
+    case LITE_ERR_CHECK: return "a kernel found a malformed Skip-List, live count or work order; outputs of that call are invalid";
     case LITE_ERR_SCRATCH_LIMIT: return "layer needs more scratch than lite_attn_fwd_noalloc's fixed 8 MiB";
     default: return "unknown status";
   }
@@ -472,6 +502,25 @@ int lite_attn_fwd(const void* q, const void* k, const void* v, void* o, float* l
   const int st = validate_fwd(a);
   if (st) return st;
   return fwd_pooled(a, nullptr, as_stream(stream));
+}
+
+int lite_attn_fwd_list(const void* q, const void* k, const void* v, void* o, float* lse, const int16_t* list,
+                       const int32_t* counts, uint32_t* mask_out, int B, int H, int N, int d, float scale, float tau,
+                       lite_stream_t stream) {
+  const FwdArgs a{q, k, v, o, lse, nullptr, mask_out, B, H, N, N, d, scale, tau};
+  int st = validate_fwd(a);
+  if (st) return st;
+  if (!list || !counts) return LITE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(list) & 1u) || (reinterpret_cast<uintptr_t>(counts) & 3u))
+    return LITE_ERR_UNSUPPORTED;
+  DeviceCache* dc = nullptr;
+  if (device_cache(&dc) != LITE_OK || ensure_pool(dc) != LITE_OK) return LITE_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  void* ws = nullptr;
+  if (cudaMallocFromPoolAsync(&ws, list_scratch_bytes(a), dc->pool, s) != cudaSuccess) return LITE_ERR_CUDA;
+  st = enqueue_list(dc, a, list, counts, static_cast<char*>(ws), s);
+  if (cudaFreeAsync(ws, s) != cudaSuccess && !st) st = LITE_ERR_CUDA;
+  return st;
 }
 
 int lite_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, const uint32_t* mask_in,

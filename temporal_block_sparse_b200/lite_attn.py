@@ -52,6 +52,7 @@ SIGNATURES = {
     "lite_mask_to_ranges": ([_P, _P, _P, _I, _I, _I, _I, _P], _I),
     "lite_set_cta_timing": ([_P, _I], _I),
     "lite_scratch_pool_bytes": ([ctypes.POINTER(ctypes.c_longlong)], _I),
+    "lite_attn_fwd_list": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _F, _P], _I),
 }
 MAX_MERGE_PARTS = 8
 
@@ -218,6 +219,35 @@ def lite_set_kernel_events(before: Optional[torch.cuda.Event], after: Optional[t
 
 def default_scale(d: int) -> float:
     return 1.0 / math.sqrt(d)
+
+
+def lite_attn_fwd_list(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lst: torch.Tensor, counts: torch.Tensor,
+                       mask_out: Optional[torch.Tensor] = None, scale: Optional[float] = None, tau: float = -10.0,
+                       o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, return_lse: bool = True,
+                       stream=None):
+    """Forward pass over caller-supplied Skip-Lists (int16 [B, H, T, T] live key tiles, descending,
+    with int32 [B, H, T] counts, as lite_mask_to_list returns them); flags are OR-ed into mask_out
+    (see include/lite_attn.h). The list buffer may be larger than [B, H, T, T]: only its first
+    B*H*T*T entries are addressed. Returns (o, lse or None)."""
+    _check_qkv(q, k, v)
+    B, N, H, d = q.shape
+    _, T, _ = lite_mask_geometry(N, d)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _check_fwd_buffers(q, k, o, lse, None, mask_out)
+    if (lst.dtype != torch.int16 or not lst.is_contiguous() or not lst.is_cuda or lst.device != q.device
+            or lst.numel() < B * H * T * T):
+        raise ValueError("lst must be a contiguous int16 CUDA tensor of at least B*H*T*T entries on q's device")
+    if (counts.dtype != torch.int32 or not counts.is_contiguous() or not counts.is_cuda or counts.device != q.device
+            or tuple(counts.shape) != (B, H, T)):
+        raise ValueError("counts must be a contiguous int32 CUDA tensor [B, H, T] on q's device")
+    st = load().lite_attn_fwd_list(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _ptr(lse), lst.data_ptr(),
+                                   counts.data_ptr(), _ptr(mask_out), B, H, N, d, float(scale or 0.0), float(tau),
+                                   _stream_handle(stream))
+    _check("lite_attn_fwd_list", st)
+    return o, lse
 
 
 def lite_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,

@@ -51,6 +51,15 @@ def test_geometry():
     assert lib.lite_mask_geometry(0, 64, None, None, None) == la.LITE_ERR_INVALID_ARG
 
 
+def test_list_entry_checks_its_arguments():
+    lib = la.load()
+    args = lambda lst, cnt: (FAKE, FAKE, FAKE, FAKE, None, lst, cnt, None, 1, 1, 256, 128, 0.0, -3.0, None)
+    assert lib.lite_attn_fwd_list(*args(None, FAKE)) == la.LITE_ERR_INVALID_ARG
+    assert lib.lite_attn_fwd_list(*args(FAKE, None)) == la.LITE_ERR_INVALID_ARG
+    assert lib.lite_attn_fwd_list(*args(FAKE + 1, FAKE)) == la.LITE_ERR_UNSUPPORTED
+    assert lib.lite_attn_fwd_list(*args(FAKE, FAKE + 2)) == la.LITE_ERR_UNSUPPORTED
+
+
 def test_scratch_pool_hook_refuses_null():
     assert la.load().lite_scratch_pool_bytes(None) == la.LITE_ERR_INVALID_ARG
 

@@ -80,7 +80,8 @@ def test_e2e_step_count():
     import bench
 
     gb = 1 << 30
-    assert bench.e2e_step_count(None, 20, 5 * gb, 600 * gb) == 20   # all fit in a third of the memory
+    assert bench.e2e_step_count(None, 20, 5 * gb, 600 * gb) == bench.E2E_DEFAULT_STEPS == 5
+    assert bench.e2e_step_count(None, 3, 5 * gb, 600 * gb) == 3     # never more than the timed steps
     assert bench.e2e_step_count(None, 20, 5 * gb, 60 * gb) == 4     # 20 GB for inputs -> 4 steps
     assert bench.e2e_step_count(None, 20, 5 * gb, 1 * gb) == 1      # never fewer than one
     assert bench.e2e_step_count(3, 20, 5 * gb, 1 * gb) == 3         # an explicit request wins

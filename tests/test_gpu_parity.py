@@ -317,3 +317,95 @@ def test_720p_layer_sampled():
 
 def test_stress_layer_sampled():
     _full_size("stress", 2, 8)
+
+
+# ------------------------------------------------- full-size workloads at their operating point
+
+
+def _mask_bits(mask, T):
+    """[B, H, Tq, W] int32 Skip-Mask -> bool [B, H, Tq, T] (True = skipped)."""
+    return np.unpackbits(mask.cpu().numpy().view(np.uint8), axis=-1, bitorder="little")[..., :T].astype(bool)
+
+
+def _lone_heavy_tiles(skipped, n, seed):
+    """Query tiles whose pair partner (2i, 2i+1 share a CTA) has a disjoint or empty live list, so
+    that the kernel's union walk gives them many key tiles computed for one query tile only; the
+    first and the ragged last tile of a head are always included."""
+    B, H, T, _ = skipped.shape
+    live = ~skipped
+    partner = np.arange(T) ^ 1
+    has_partner = partner < T
+    own = live.sum(-1)
+    shared = np.where(has_partner, (live & live[:, :, np.minimum(partner, T - 1)]).sum(-1), 0)
+    lone = own - shared  # live tiles of this query tile that its partner skips
+    rng = np.random.default_rng(seed)
+    picks = {(0, 0, 0), (B - 1, H - 1, T - 1)}
+    if (~has_partner).any():
+        picks.add((0, int(rng.integers(H)), T - 1))  # an unpaired last tile
+    order = np.argsort(-(lone + rng.random(lone.shape)), axis=None)  # most lone tiles first, ties random
+    for flat in order[: 4 * n]:
+        b, h, i = np.unravel_index(flat, lone.shape)
+        picks.add((int(b), int(h), int(i)))
+        if len(picks) >= n - 2:
+            break
+    empty_partner = np.argwhere((own > 0) & has_partner & (own[:, :, np.minimum(partner, T - 1)] == 0))
+    for b, h, i in empty_partner[:2]:
+        picks.add((int(b), int(h), int(i)))
+    while len(picks) < n:
+        picks.add((int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(T))))
+    frac_lone = float(lone.sum() / max(own.sum(), 1))
+    return sorted(picks), frac_lone
+
+
+def _operating_point(name, advance, n_compare, n_tiles, min_skipped):
+    """Advance a workload's trajectory on the GPU alone for `advance` steps (its own tau schedule,
+    the Skip-Mask growing step to step in the benchmark's launch configuration), then compare the
+    next `n_compare` steps with the oracle, teacher-forced on the GPU's mask_in, on sampled query
+    tiles biased to lone union tiles."""
+    w = wl.WORKLOADS[name]
+    tr = wl.Trajectory(w, device="cuda")
+    B, N, H, d = w.B, w.N, w.H, w.d
+    _, T, _ = la.lite_mask_geometry(N, d)
+    m_in = la.new_mask(B, H, N, d)
+    m_out = torch.empty_like(m_in)
+    o = torch.empty((B, N, H, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    for t in range(advance):
+        q, k, v = tr.current()
+        la.lite_attn_fwd(q, k, v, m_in, m_out, tau=w.tau(t), o=o, lse=lse)
+        m_in, m_out = m_out, m_in
+        tr.advance()
+    assert la.lite_get_device_status() == 0
+    for t in range(advance, advance + n_compare):
+        q, k, v = tr.current()
+        skipped = _mask_bits(m_in, T)
+        frac = float(skipped.mean())
+        assert frac >= min_skipped, (name, t, frac)
+        tiles, lone = _lone_heavy_tiles(skipped, n_tiles, seed=t)
+        la.lite_attn_fwd(q, k, v, m_in, m_out, tau=w.tau(t), o=o, lse=lse)
+        assert la.lite_get_device_status() == 0
+        ref = oracle_step(q, k, v, m_in, w.tau(t), query_tiles=tiles)
+        rep = compare(o, lse, m_out, ref)
+        assert_within(rep)
+        grown = _mask_bits(m_out, T)
+        assert (grown | ~skipped).all()  # monotone: every skipped tile stays skipped
+        print(f"{name} step {t}: skipped {frac:.3f}, lone share of live tiles {lone:.3f}, "
+              f"flagged(sampled) {rep.flagged}, near-tau mismatches {rep.mask_mismatches}, "
+              f"o_max {rep.o_max_abs:.2e} rel_rms {rep.o_rel_rms:.2e} lse {rep.lse_max_abs:.2e}")
+        m_in, m_out = m_out, m_in
+        tr.advance()
+
+
+def test_720p_layer_after_ten_steps():
+    """The 720p layer (tau -3) once half of its tiles are skipped."""
+    _operating_point("720p", 10, 2, 16, 0.5)
+
+
+def test_stress_layer_after_twelve_steps():
+    """The stress layer (B=2, per-head locality U[2,8]) at >= 75% skipped, with its per-head spread."""
+    _operating_point("stress", 12, 2, 20, 0.75)
+
+
+def test_480p_layer_last_step_of_its_schedule():
+    """Step 9, the last of the 480p schedule (tau 0)."""
+    _operating_point("480p", 9, 1, 16, 0.3)
