@@ -13,17 +13,14 @@
 // Warp roles (320 threads):
 //   warp 0       TMA producer: per item the pair's two Q tiles; per union tile u a load bundle with
 //                K_u (2-stage ring) and V_{u-1} (2-stage ring), one barrier per bundle. It walks the
-//                two lists, checks them (in range, strictly descending; a bad list or count stops
-//                the kernel with LITE_ERR_CHECK in the status word), assigns each computed tile one
-//                of the two TMEM score buffers, and hands the MMA thread, per union tile, for which
-//                query tiles it is live and in which buffer (a small shared-memory ring written
-//                before the bundle is armed), and each softmax group a descriptor per tile of its
-//                query tile (key tile, buffer) through a ring of its own.
+//                two lists, checks them (in range, strictly descending; a bad list, live count or
+//                work-order entry stops the kernel with LITE_ERR_CHECK in the status word), and
+//                hands the MMA thread, per union tile, which query tiles it is live for, in a small
+//                shared-memory ring written before the bundle is armed.
 //   warp 1       TMEM allocator and single-thread tcgen05 MMA issuer. Per union tile u, for query
-//                tile g = 0, 1: QK_g(u) into a free score buffer if one is free, then PV_g(u-1) if
-//                u-1 was live for g, then QK_g(u) if it had to wait for that buffer:
-//                  S = Q_g K_u^T     (SS form) into score buffer b,
-//                  O_g += P V_{u-1}  (TS form: P read from the buffer it was written to).
+//                tile g = 0, 1: PV_g(u-1) if u-1 was live for g, then QK_g(u) if u is live for g:
+//                  S_g = Q_g K_u^T    (SS form) into TMEM buffer g,
+//                  O_g += P_g V_{u-1} (TS form: P read from TMEM, V from shared memory).
 //   warps 2..5   softmax warpgroup 0, query tile 0 of the pair; warps 6..9: group 1, query tile 1.
 //                One thread per query row (TMEM lane). Per live tile of its query tile: row max;
 //                the QK-Skip vote (skill page "Lite Attention Temporal Sparse", Core Concept: a
@@ -34,14 +31,9 @@
 //                kRescaleLog2. The two groups run on the two query tiles at once, so the latency of
 //                one hides the other's.
 //
-// Score buffers. The two TMEM score buffers belong to no group: a tile's S (then its P) occupies a
-// buffer from its QK until its PV has been issued. Where both query tiles are live on consecutive
-// union tiles each keeps one buffer. Where a key tile is live for one query tile only (the lists of
-// neighbouring query tiles differ), that group's next QK goes into the buffer its partner is not
-// using, ahead of the PV of its current tile, so one group keeps two tiles in flight and its softmax
-// never waits for its own QK; and a QK whose buffer is free is issued before any PV that waits for
-// a softmax, so lone tiles of the two groups overlap.
-//
+// Every wait is bounded by a wall-clock limit; on expiry the kernel records a timeout in the device
+// status word, every role stops, in-flight copies and MMAs are drained, TMEM is freed and the CTA
+// exits. No trap, no unbounded spin.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -118,7 +110,7 @@ struct AttnCfg {
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;
   static constexpr int OFF_CTL = OFF_V + 2 * KV_BYTES;
-  static constexpr int CTL_BYTES = 1024;
+  static constexpr int CTL_BYTES = 512;
   // O staging for the TMA stores of the epilogue: per softmax warp, 16 rows of D columns, as
   // NCHUNK 128-byte-swizzled panels of 16 x 128 bytes (1024-aligned)
   static constexpr int OST_ROWS = 16;
@@ -163,36 +155,23 @@ constexpr uint32_t kLast0 = 16u, kLast1 = 32u;      // last live tile of query t
 constexpr uint32_t kItemFirst = 64u;                // first union tile of an item
 constexpr uint32_t kItemLast = 128u;                // last union tile of an item
 constexpr uint32_t kEnd = 256u;                     // no more tiles (the bundle carries the last V)
-constexpr uint32_t kItemOdd = 512u, kItemAfterFirst = 1024u;  // item parity, "not the CTA's first item"
-constexpr int kBufShift = 11;                       // bit 11 + g: QK_g(u) goes to score buffer 1 (else 0)
-constexpr int kEarlyShift = 13;                     // bit 13 + g: QK_g(u) is issued before the PVs of u
-
-// Per tile of a query tile, what the producer tells its softmax group (one 32-bit word in a ring of
-// kDescRing slots per group): the list entry (key tile and its no-flag tag), the score buffer, and
-// whether the tile's QK was issued before the PV of the group's previous tile (borrowed buffer).
-constexpr int kDescRing = 8;
-constexpr int kDescBufShift = 16;
-constexpr uint32_t kDescBorrowed = 1u << 17;
+constexpr int kItemShift = 12;                      // bits 12..31: the item's number in this CTA
 
 // Control block in shared memory (barriers are 8-byte mbarrier objects).
 struct alignas(8) AttnCtl {
   uint64_t q_full, q_empty;          // the pair's Q tiles landed / read by the item's last QK
   uint64_t kv_full[2];               // bundle u landed: K_u (stage u%2) and V_{u-1} (stage (u-1)%2)
   uint64_t kv_free[2];               // the QKs of union tile u (and every MMA before them) finished
-  uint64_t s_full[2][2];             // [g][b]: S of group g's tile ready in buffer b (a phase per use of b by g)
-  uint64_t p_full[2];                // [b]: P written into buffer b (a phase per occupancy of b)
-  uint64_t pv_o[2];                  // [g]: the PV before a borrowed tile of g finished (a phase per such tile)
+  uint64_t s_full[2];                // S_g ready (one phase per live tile of query tile g)
+  uint64_t p_full[2];                // P_g written (one phase per live tile of query tile g)
   uint64_t pv_done[2];               // last PV_g of an item finished (accumulator g)
   uint64_t o_free[2];                // group g's epilogue has read O_g (one phase per item)
   uint64_t item_full[2], item_empty[2];
-  uint64_t desc_full[2][kDescRing];  // descriptor slot written (a phase per kDescRing tiles of the group)
-  uint64_t desc_empty[2][kDescRing]; // descriptor slot read by the group's four warps
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
   uint32_t tiles;                    // live (query tile, key tile) pairs processed (measurement hook)
   uint32_t ring[4];                  // per union tile u (slot u%4): the flags above
-  uint32_t desc[2][kDescRing];       // per group: tile descriptors
   PairInfo info[2];                  // handed-out items
 };
 // UMMA shared-memory descriptor, 128-byte swizzle (layout type 2, bits 61-63), version 1 (bit 46).
@@ -268,7 +247,6 @@ struct Waiter {
     return true;
   }
   __device__ __forceinline__ void give_up() const { stop(kStatusTimeout); }
-  // A consistency check failed: record it and make every role stop at its next wait.
   __device__ __forceinline__ void fail_check() const { stop(kStatusCheck); }
   __device__ __forceinline__ void stop(int code) const {
     *abort = 1;
@@ -342,6 +320,9 @@ struct ListCursor {
 // exact running max within ~1% of the speed of 8.
 constexpr float kRescaleLog2 = 2.0f;
 
+// Item parity and "not the CTA's first item" travel in the ring word next to the tile flags.
+constexpr uint32_t kItemOdd = 512u, kItemAfterFirst = 1024u;
+
 template <int D, int BN>
 __global__ void __launch_bounds__(320, 1)
     lite_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -367,18 +348,12 @@ __global__ void __launch_bounds__(320, 1)
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(BAR(kv_full[b]), 1);
       ptx::mbar_init(BAR(kv_free[b]), 1);
-      ptx::mbar_init(BAR(s_full[0][b]), 1);
-      ptx::mbar_init(BAR(s_full[1][b]), 1);
+      ptx::mbar_init(BAR(s_full[b]), 1);
       ptx::mbar_init(BAR(p_full[b]), 128);
-      ptx::mbar_init(BAR(pv_o[b]), 1);
       ptx::mbar_init(BAR(pv_done[b]), 1);
       ptx::mbar_init(BAR(o_free[b]), 128);
       ptx::mbar_init(BAR(item_full[b]), 1);
       ptx::mbar_init(BAR(item_empty[b]), 8);  // one lane of each softmax warp
-      for (int x = 0; x < kDescRing; ++x) {
-        ptx::mbar_init(BAR(desc_full[b][x]), 1);
-        ptx::mbar_init(BAR(desc_empty[b][x]), 4);  // one lane of each warp of group b
-      }
     }
     ptx::mbar_init(BAR(drain), 1);
     ctl->abort = 0;
@@ -409,21 +384,17 @@ __global__ void __launch_bounds__(320, 1)
   const Waiter wt{&ctl->abort, p.status, p.wait_limit_ns};
 
   // Barrier phases. Union tiles u are numbered over all items this CTA processes; bundle u uses
-  // kv_full / kv_free slot u%2 and ring slot u%4. An occupancy of score buffer b is one tile's S and
-  // P in it, from its QK to its PV; s_full[g][b] completes once per occupancy of b by group g's
-  // tiles, p_full[b] once per occupancy of b, pv_o[g] once per borrowed tile of g, desc_full and
-  // desc_empty of slot x of group g once per kDescRing tiles of g; q_full / q_empty and o_free[g]
-  // once per item with tiles, pv_done[g] once per item in which query tile g has a live tile.
-  // Every waiter either observes each phase of a barrier in order, or the order of the MMA thread's
-  // commits keeps the barrier within one phase of the awaited one (the argument is written at each
-  // wait), so the parity waits are exact.
+  // kv_full / kv_free slot u%2 and ring slot u%4. s_full[g] and p_full[g] complete once per live
+  // tile of query tile g, q_full / q_empty and o_free[g] once per item with tiles, pv_done[g] once
+  // per item in which query tile g has a live tile. Every waiter either observes each phase of a
+  // barrier in order, or the order of the MMA thread's commits keeps the barrier within one phase
+  // of the awaited one (the argument is written at each wait), so the parity waits are exact.
   if (warp == 0) {
     // ------------------------------------------------------------------------- TMA producer
     // Bundle u carries K_u (stage u%2) and V_{u-1} (stage (u-1)%2). K stage u%2 was last read by
     // the QKs of union tile u-2; V stage (u-1)%2 by the PVs of union tile u-3, which the MMA thread
-    // issues before the end of union tile u-2, whose commit frees the bundle. So one wait (kv_free
-    // of u-2) frees both, and the MMA thread waits once per union tile. A last bundle carries only
-    // the final V, with the end mark.
+    // issues before those QKs. So one wait (kv_free of u-2) frees both, and the MMA thread waits
+    // once per union tile. A last bundle carries only the final V, with the end mark.
     if (lane == 0) {
       uint32_t u = 0, items = 0, qn = 0, live_pairs = 0;
       bool ok = true;
@@ -431,11 +402,7 @@ __global__ void __launch_bounds__(320, 1)
       bool q_armed = false, kv_armed[2] = {false, false};
       uint32_t q_par = 0, kv_par[2] = {0, 0};
       int pj = 0, ph = 0, pb = 0;  // coordinates of union tile u-1
-      // score-buffer state: pend[g] = buffer holding group g's tile of union tile u-1 (its PV is
-      // issued during union tile u), -1 if g was not live there
-      int pend[2] = {-1, -1};
-      bool v_needed = false;        // union tile u-1 had a live tile, so bundle u carries V_{u-1}
-      uint32_t dcount[2] = {0, 0};  // descriptors posted per group
+      bool v_needed = false;       // union tile u-1 had a live tile, so bundle u carries V_{u-1}
       // kv_free of slot u%2 next completes with the QKs of union tile u, which need this bundle
       auto bundle = [&](bool with_k, int j, int h, int b, uint32_t flags) -> bool {
         LITE_TRACE(0, 0, u);
@@ -455,17 +422,6 @@ __global__ void __launch_bounds__(320, 1)
         ph = h;
         pb = b;
         ++u;
-        return true;
-      };
-      // Descriptor of group g's next tile. Slot c % kDescRing is rewritten only after the group's
-      // four warps read its previous content (desc_empty, one phase per kDescRing tiles; exact:
-      // the group cannot release a slot twice before the producer fills it again).
-      auto post = [&](int g, int entry, int buf, bool borrowed) -> bool {
-        const uint32_t c = dcount[g], slot = c % kDescRing;
-        if (c >= kDescRing && !wt.wait(BAR(desc_empty[g][slot]), ((c / kDescRing) - 1) & 1)) return false;
-        ctl->desc[g][slot] = uint32_t(entry & 0xffff) | (uint32_t(buf) << kDescBufShift) | (borrowed ? kDescBorrowed : 0u);
-        ptx::mbar_arrive(BAR(desc_full[g][slot]));  // release: the group reads the word after its wait
-        dcount[g] = c + 1;
         return true;
       };
       while (ok) {
@@ -495,10 +451,7 @@ __global__ void __launch_bounds__(320, 1)
           // thread issues with the next bundle; and before this producer hands out two more items,
           // both groups must have read this one. So the pending PVs are flushed now, by a bundle
           // with V only and no live tile.
-          if (pend[0] >= 0 || pend[1] >= 0) {
-            ok = bundle(false, 0, 0, 0, 0u);
-            pend[0] = pend[1] = -1;
-          }
+          if (v_needed) ok = bundle(false, 0, 0, 0, 0u);
           continue;
         }
         // the pair's Q tiles; q_empty is committed after the item's last QK
@@ -512,71 +465,26 @@ __global__ void __launch_bounds__(320, 1)
         q_armed = true;
         q_par = qn & 1;
         // the union of the two descending lists, highest key tile first
-        ListCursor cur[2] = {{it.row0, it.n[0], 0, it.e[0][0], it.e[0][1], p.Tk},
-                             {it.row0 + 1, it.n[1], 0, it.e[1][0], it.e[1][1], p.Tk}};
+        ListCursor c0{it.row0, it.n[0], 0, it.e[0][0], it.e[0][1], p.Tk};
+        ListCursor c1{it.row0 + 1, it.n[1], 0, it.e[1][0], it.e[1][1], p.Tk};
         const uint32_t item_bits = ((qn & 1) ? kItemOdd : 0u) | (qn >= 1 ? kItemAfterFirst : 0u);
         uint32_t f = kItemFirst;
         while (ok) {
-          const int j = max(cur[0].head(), cur[1].head());
-          bool live[2];
-          int ent[2];
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            live[g] = cur[g].head() == j;
-            ent[g] = cur[g].cur;
-            if (live[g] && !cur[g].head_ok()) ok = false;  // malformed or not descending
-          }
-          if (!ok) {
-            wt.fail_check();
+          const int h0 = c0.head(), h1 = c1.head();
+          const int j = max(h0, h1);
+          if ((h0 == j && !c0.head_ok()) || (h1 == j && !c1.head_ok())) {
+            wt.fail_check();  // malformed or not strictly descending
+            ok = false;
             break;
           }
           f |= item_bits;
-#pragma unroll
-          for (int g = 0; g < 2; ++g)
-            if (live[g])
-              f |= (kLive0 << g) | (cur[g].i == 0 ? (kFirst0 << g) : 0u) | (cur[g].i == cur[g].n - 1 ? (kLast0 << g) : 0u);
-#pragma unroll
-          for (int g = 0; g < 2; ++g)
-            if (live[g]) cur[g].advance(p);
-          const bool last = cur[0].head() < 0 && cur[1].head() < 0;
+          if (h0 == j) f |= kLive0 | (c0.i == 0 ? kFirst0 : 0u) | (c0.i == c0.n - 1 ? kLast0 : 0u);
+          if (h1 == j) f |= kLive1 | (c1.i == 0 ? kFirst1 : 0u) | (c1.i == c1.n - 1 ? kLast1 : 0u);
+          if (h0 == j) c0.advance(p);
+          if (h1 == j) c1.advance(p);
+          const bool last = c0.head() < 0 && c1.head() < 0;
           if (last) f |= kItemLast;
-          // Score buffers, in the MMA thread's issue order. First every QK whose buffer is free now
-          // (for a group with a tile in flight, the buffer it does not hold: a borrowed buffer);
-          // then, per group, the PV of its previous tile, which frees that tile's buffer, and the
-          // QKs that waited for it.
-          uint32_t held = (pend[0] >= 0 ? 1u << pend[0] : 0u) | (pend[1] >= 0 ? 1u << pend[1] : 0u);
-          int qb[2] = {-1, -1};
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            if (!live[g]) continue;
-            int c = pend[g] >= 0 ? 1 - pend[g] : g;
-            if ((held >> c) & 1u) c = pend[g] >= 0 ? -1 : 1 - g;
-            if (c >= 0 && !((held >> c) & 1u)) {
-              qb[g] = c;
-              held |= 1u << c;
-              f |= 1u << (kEarlyShift + g);
-            }
-          }
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            if (pend[g] >= 0) held &= ~(1u << pend[g]);
-            if (live[g] && qb[g] < 0) {
-              const int c = (pend[g] >= 0 && !((held >> pend[g]) & 1u)) ? pend[g] : (((held >> g) & 1u) ? 1 - g : g);
-              qb[g] = c;
-              held |= 1u << c;
-            }
-          }
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            if (live[g]) {
-              f |= uint32_t(qb[g]) << (kBufShift + g);
-              const bool borrowed = ((f >> (kEarlyShift + g)) & 1u) && pend[g] >= 0;
-              if (ok) ok = post(g, ent[g], qb[g], borrowed);
-            }
-          }
-          pend[0] = live[0] ? qb[0] : -1;
-          pend[1] = live[1] ? qb[1] : -1;
-          if (ok) ok = bundle(true, j, it.h, it.b, f);
+          ok = bundle(true, j, it.h, it.b, f);
           if (last) break;
           f = 0u;
         }
@@ -594,15 +502,14 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------------- MMA issuer
-    // Per union tile u, once bundle u landed: first the QKs the producer marked early (their score
-    // buffer is free now), then for g = 0, 1: PV_g(u-1) if u-1 was live for query tile g, and
-    // QK_g(u) if it was not early (it reuses the buffer that PV just read). MMAs of this thread run
-    // in issue order, so a QK into a buffer always follows the PV that read the P in it. One commit
-    // per union tile frees the bundle's stages.
+    // Per union tile u, once bundle u landed: for g = 0, 1, PV_g(u-1) if u-1 was live for query
+    // tile g, then QK_g(u) if u is live for it. QK_g(u) reuses S buffer g after PV_g(u-1) read the
+    // P in it, and the next QK_g needs the softmax's P_g of this tile first: MMAs of this thread
+    // run in issue order. One commit per union tile frees the bundle's stages.
     if (lane == 0) {
       uint32_t u = 0;
-      uint32_t pvk[2] = {0, 0};  // PVs issued per score buffer (= P phases consumed per buffer)
-      uint32_t prev = 0;         // flags of union tile u-1
+      uint32_t pc[2] = {0, 0};  // P phases consumed per query tile
+      uint32_t prev = 0;        // flags of union tile u-1
       bool ok = true;
       // 128B-swizzled K-major operands advance 32 bytes (>> 4 = 2) per K=16 step inside an atom;
       // V (MN-major) advances 16 rows = 2048 bytes (>> 4 = 128) per step.
@@ -627,52 +534,25 @@ __global__ void __launch_bounds__(320, 1)
         ptx::tc_fence_after();
         // q_full completes once per item; the next load waits for this item's q_empty commit
         bool need_q = (f & kItemFirst) != 0u;
-        const uint64_t kd = k_desc0 + uint64_t(((u & 1) * C::KV_BYTES) >> 4);
-        // S = Q_g K_u^T into the buffer the producer assigned. s_full[g][b] completes once per use
-        // of buffer b by group g; the group waits for its uses in order, and the next use of b
-        // needs a PV after the group's P of this one, so the group is never a phase behind.
-        auto qk = [&](int g) -> bool {
-          if (need_q) {
-            if (!wt.wait(BAR(q_full), (f & kItemOdd) ? 1u : 0u)) return false;
-            ptx::tc_fence_after();
-            need_q = false;
-          }
-          const int b = int((f >> (kBufShift + g)) & 1u);
-          const uint64_t qd = q_desc0 + uint64_t((g * C::Q_BYTES) >> 4);
-          const uint32_t s_tmem = tmem + C::S_COL + b * BN;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = uint64_t((kk >> 2) * (C::Q_CHUNK >> 4) + (kk & 3) * 2);
-            const uint64_t offk = uint64_t((kk >> 2) * (C::KV_CHUNK >> 4) + (kk & 3) * 2);
-            ptx::mma_ss(s_tmem, qd + off, kd + offk, C::IDESC_QK, kk > 0 ? 1u : 0u);
-          }
-          ptx::mma_commit(BAR(s_full[g][b]));
-          return true;
-        };
-#pragma unroll
-        for (int g = 0; g < 2; ++g)
-          if ((f & (kLive0 << g)) && ((f >> (kEarlyShift + g)) & 1u) && !qk(g)) ok = false;
-        if (!ok) break;
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
           if (prev & (kLive0 << g)) {
             // The first PV of query tile g in an item overwrites O_g: the previous item's epilogue
             // of group g must have read it (o_free[g]: one phase per item, exact because the next
-            // phase needs this item's PVs). p_full[b] next completes for the next occupancy of b,
-            // whose S needs a QK issued after this PV.
+            // phase needs this item's PVs). p_full[g] next completes for g's next live tile, whose
+            // S needs a QK issued after this PV.
             if ((prev & (kFirst0 << g)) && (prev & kItemAfterFirst) &&
                 !wt.wait(BAR(o_free[g]), (prev & kItemOdd) ? 0u : 1u)) {
               ok = false;
               break;
             }
-            const int b = int((prev >> (kBufShift + g)) & 1u);
-            if (!wt.wait(BAR(p_full[b]), pvk[b] & 1)) {
+            if (!wt.wait(BAR(p_full[g]), pc[g] & 1)) {
               ok = false;
               break;
             }
-            ++pvk[b];
+            ++pc[g];
             ptx::tc_fence_after();
-            const uint32_t p_tmem = tmem + C::S_COL + b * BN;
+            const uint32_t p_tmem = tmem + C::S_COL + g * BN;
             const uint32_t o_tmem = tmem + C::O_COL + g * D;
             const uint64_t vd = v_desc0 + uint64_t((((u - 1) & 1) * C::KV_BYTES) >> 4);
             const bool fresh = (prev & (kFirst0 << g)) != 0u;
@@ -681,13 +561,26 @@ __global__ void __launch_bounds__(320, 1)
               ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + uint64_t(kk * 128), C::IDESC_PV, (fresh && kk == 0) ? 0u : 1u);
             // the epilogue of group g waits for the item's last PV into its accumulator
             if (prev & (kLast0 << g)) ptx::mma_commit(BAR(pv_done[g]));
-            // a tile of g whose QK went ahead of this PV (borrowed buffer) may rescale O_g only
-            // once this PV has finished
-            if ((f & (kLive0 << g)) && ((f >> (kEarlyShift + g)) & 1u)) ptx::mma_commit(BAR(pv_o[g]));
           }
-          if ((f & (kLive0 << g)) && !((f >> (kEarlyShift + g)) & 1u) && !qk(g)) {
-            ok = false;
-            break;
+          if (f & (kLive0 << g)) {
+            if (need_q) {
+              if (!wt.wait(BAR(q_full), (f & kItemOdd) ? 1u : 0u)) {
+                ok = false;
+                break;
+              }
+              ptx::tc_fence_after();
+              need_q = false;
+            }
+            const uint64_t qd = q_desc0 + uint64_t((g * C::Q_BYTES) >> 4);
+            const uint64_t kd = k_desc0 + uint64_t(((u & 1) * C::KV_BYTES) >> 4);
+            const uint32_t s_tmem = tmem + C::S_COL + g * BN;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t off = uint64_t((kk >> 2) * (C::Q_CHUNK >> 4) + (kk & 3) * 2);
+              const uint64_t offk = uint64_t((kk >> 2) * (C::KV_CHUNK >> 4) + (kk & 3) * 2);
+              ptx::mma_ss(s_tmem, qd + off, kd + offk, C::IDESC_QK, kk > 0 ? 1u : 0u);
+            }
+            ptx::mma_commit(BAR(s_full[g]));
           }
         }
         LITE_TRACE(1, 2, u);
@@ -715,8 +608,6 @@ __global__ void __launch_bounds__(320, 1)
     const int wrow = quarter * 32 - grp * C::ROW1;
     const bool idle_warp = C::ROW1 > 0 && (wrow < 0 || wrow >= C::BQ);
     uint32_t tg = 0, items = 0, pv_phase = 0;
-    uint32_t uses[2] = {0, 0};  // this group's tiles so far in score buffer 0 / 1 (s_full[grp][b] phases)
-    uint32_t borrowed_n = 0;    // this group's borrowed tiles so far (pv_o[grp] phases)
     while (true) {
       const int slot = items & 1;
       bool ok = wt.wait(BAR(item_full[slot]), (items >> 1) & 1);
@@ -746,28 +637,21 @@ __global__ void __launch_bounds__(320, 1)
       float m_true = -INFINITY;  // running max over the tile's earlier live key tiles (log2 units)
       float m_used = -INFINITY;  // exponent reference (lazy rescale)
       float l = 0.f;             // row sum relative to m_used
+      int e_cur = it.e[grp][0], e_nxt = it.e[grp][1];
       for (int idx = 0; idx < n; ++idx) {
         const uint32_t t = tg + idx;
-        // this tile's descriptor: slot t % kDescRing, one desc_full phase per kDescRing tiles of the
-        // group (exact: the producer refills a slot only after the group's four warps read it)
-        const uint32_t dslot = t % kDescRing;
-        wt.wait(BAR(desc_full[grp][dslot]), (t / kDescRing) & 1);
-        const uint32_t dsc = ctl->desc[grp][dslot];
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(BAR(desc_empty[grp][dslot]));
-        const int j = int(dsc & kListIndexMask);
-        const bool may_flag = !(dsc & kListNoFlag);
-        const int sb = int((dsc >> kDescBufShift) & 1u);  // score buffer of this tile
-        const bool borrowed = (dsc & kDescBorrowed) != 0u;
+        const int j = e_cur & kListIndexMask;
+        const bool may_flag = !(e_cur & kListNoFlag);
+        e_cur = e_nxt;
+        if (idx + 2 < n) e_nxt = key_entry(p, row, idx + 2);  // prefetch
         if (r == 0) LITE_TRACE(2 + grp, 0, t);
-        // s_full[grp][sb] next completes for this group's next use of buffer sb
-        wt.wait(BAR(s_full[grp][sb]), uses[sb] & 1);
-        ++uses[sb];
+        // s_full[g] next completes for g's next live tile, whose QK follows this tile's PV
+        wt.wait(BAR(s_full[grp]), t & 1);
         __syncwarp();
         ptx::tc_fence_after();
         float loc = -INFINITY;  // the tile's row max (log2 units)
         if (!idle_warp) {
-        const uint32_t s_tmem = tmem + lane_base + C::S_COL + sb * BN;
+        const uint32_t s_tmem = tmem + lane_base + C::S_COL + grp * BN;
         // the whole S row is read once and stays in registers for the max and the exponentials
         uint32_t sr[BN];
 #pragma unroll
@@ -795,11 +679,8 @@ __global__ void __launch_bounds__(320, 1)
         }
         loc = ptx::fmax3(m0, m1, fmaxf(m2, m3)) * p.scale_log2;
         // lazy rescale of the accumulator: move the reference only when the tile max exceeds it by
-        // more than kRescaleLog2. Unless this tile's buffer was borrowed, the previous PV into O_g
-        // was issued before this tile's QK, so it has completed now that S is ready; a borrowed
-        // tile's QK went ahead of that PV, whose completion pv_o[grp] signals (one phase per
-        // borrowed tile; exact: the next phase needs this tile's P). The rescaled O is stored
-        // before P is released.
+        // more than kRescaleLog2. The previous PV into O_g was issued before this tile's QK, so it
+        // has completed now that S is ready; the rescaled O is stored before P is released.
         const bool need = loc > m_used + kRescaleLog2;
         float alpha = 1.f;
         if (need) {
@@ -808,10 +689,6 @@ __global__ void __launch_bounds__(320, 1)
           l *= alpha;
         }
         if (__any_sync(0xffffffffu, need) && idx >= 1) {
-          if (borrowed) {
-            wt.wait(BAR(pv_o[grp]), borrowed_n & 1);
-            ptx::tc_fence_after();
-          }
           const uint32_t o_tmem = tmem + lane_base + C::O_COL + grp * D;
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
@@ -847,9 +724,8 @@ __global__ void __launch_bounds__(320, 1)
         const float2 acc2 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
         l += acc2.x + acc2.y;
         }
-        if (borrowed) ++borrowed_n;
         ptx::tc_fence_before();
-        ptx::mbar_arrive(BAR(p_full[sb]));
+        ptx::mbar_arrive(BAR(p_full[grp]));
         if (r == 0) LITE_TRACE(2 + grp, 2, t);
         if (p.skip_test) {
           // QK-Skip, off the path from S to P: flag key tile j when loc - m < tau for every valid

@@ -409,3 +409,30 @@ def test_stress_layer_after_twelve_steps():
 def test_480p_layer_last_step_of_its_schedule():
     """Step 9, the last of the 480p schedule (tau 0)."""
     _operating_point("480p", 9, 1, 16, 0.3)
+
+
+def test_two_empty_items_after_a_full_one():
+    """One CTA, work items in their natural order: a pair of query tiles with live key tiles, then
+    two pairs whose query tiles are fully skipped, then live pairs again. The producer must release
+    the first pair's last PV before it hands out more items (a bundle with V only); without that
+    the CTA stalls until the wait limit, which is lowered here so that a stall shows as
+    LITE_ERR_TIMEOUT within half a second."""
+    w = wl.small_workload(1, 2, 2, 8, 64, 128, steps=1, locality=3.0, tau=-2.0, seed_offset=71)  # N=1024, T=8
+    q, k, v = wl.Trajectory(w, device="cuda").current()
+    B, N, H, d = q.shape
+    _, T, W = la.lite_mask_geometry(N, d)
+    assert T == 8 and W == 1
+    mask = la.new_mask(B, H, N, d)
+    mask[:, :, 2:6, 0] = (1 << T) - 1  # query tiles 2..5 (pairs 1 and 2) skip every key tile
+    m_out = torch.empty_like(mask)
+    la.lite_set_option(la.LITE_OPT_MAX_CTAS, 1)
+    la.lite_set_option(la.LITE_OPT_SCHEDULE, 0)
+    la.lite_set_option(la.LITE_OPT_WAIT_LIMIT_NS, 500_000_000)
+    try:
+        o, lse = la.lite_attn_fwd(q, k, v, mask, m_out, tau=-2.0)
+        assert la.lite_get_device_status() == 0
+    finally:
+        la.lite_set_option(la.LITE_OPT_SCHEDULE, 1)
+    rep = compare(o, lse, m_out, oracle_step(q, k, v, mask, -2.0))
+    assert_within(rep)
+    assert torch.isneginf(lse[:, :, 2 * 128:6 * 128]).all()
