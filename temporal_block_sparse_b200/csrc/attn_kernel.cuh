@@ -679,26 +679,14 @@ __global__ void __launch_bounds__(320, 1)
         }
         loc = ptx::fmax3(m0, m1, fmaxf(m2, m3)) * p.scale_log2;
         // lazy rescale of the accumulator: move the reference only when the tile max exceeds it by
-        // more than kRescaleLog2. The previous PV into O_g was issued before this tile's QK, so it
-        // has completed now that S is ready; the rescaled O is stored before P is released.
+        // more than kRescaleLog2. O itself is rescaled after the exponentials below, when the S row
+        // no longer occupies registers (doing it here made the compiler spill S on every tile).
         const bool need = loc > m_used + kRescaleLog2;
         float alpha = 1.f;
         if (need) {
           alpha = ptx::ex2(m_used - loc);
           m_used = loc;
           l *= alpha;
-        }
-        if (__any_sync(0xffffffffu, need) && idx >= 1) {
-          const uint32_t o_tmem = tmem + lane_base + C::O_COL + grp * D;
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t rr[32];
-            ptx::tmem_ld32(o_tmem + c * 32, rr);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int x = 0; x < 32; ++x) rr[x] = __float_as_uint(__uint_as_float(rr[x]) * alpha);
-            ptx::tmem_st32(o_tmem + c * 32, rr);
-          }
         }
         // P = 2^(s*scale*log2e - m_used) as bf16 pairs over the S columns (chunk c of 32 key
         // columns -> TMEM columns [16c, 16c+16)), released to the MMA thread in one piece. Packed
@@ -719,6 +707,20 @@ __global__ void __launch_bounds__(320, 1)
             pk[x] = *reinterpret_cast<uint32_t*>(&h2);
           }
           ptx::tmem_st16(s_tmem + c * 16, pk);
+        }
+        // The previous PV into O_g was issued before this tile's QK, so it has completed now that S
+        // is ready; the rescaled O is stored before P is released (both stores are waited for below).
+        if (__any_sync(0xffffffffu, need) && idx >= 1) {
+          const uint32_t o_tmem = tmem + lane_base + C::O_COL + grp * D;
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t rr[32];
+            ptx::tmem_ld32(o_tmem + c * 32, rr);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) rr[x] = __float_as_uint(__uint_as_float(rr[x]) * alpha);
+            ptx::tmem_st32(o_tmem + c * 32, rr);
+          }
         }
         ptx::tmem_wait_st();
         const float2 acc2 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
