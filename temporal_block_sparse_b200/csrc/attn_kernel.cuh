@@ -26,7 +26,7 @@
 //                the QK-Skip vote (skill page "Lite Attention Temporal Sparse", Core Concept: a
 //                tile whose local max score is far below the cumulative max is flagged) against
 //                the running max over the tile's earlier live tiles; one atomicOr per flagged
-//                (query tile, key tile); exp2 (an eighth on the FMA pipe); P (bf16) back into TMEM
+//                (query tile, key tile); exp2 (a sixteenth on the FMA pipe); P (bf16) back into TMEM
 //                over the consumed S columns; O rescale when the reference max grew by more than
 //                kRescaleLog2. The two groups run on the two query tiles at once, so the latency of
 //                one hides the other's.
@@ -690,8 +690,9 @@ __global__ void __launch_bounds__(320, 1)
         }
         // P = 2^(s*scale*log2e - m_used) as bf16 pairs over the S columns (chunk c of 32 key
         // columns -> TMEM columns [16c, 16c+16)), released to the MMA thread in one piece. Packed
-        // fp32x2 arithmetic for the affine step and the row sum; one column pair in eight is
-        // exponentiated on the FMA pipe, the rest on MUFU (the share that balanced the two best).
+        // fp32x2 arithmetic for the affine step and the row sum; one column pair in sixteen is
+        // exponentiated on the FMA pipe, the rest on MUFU (measured: 1/16 and none beat 1/8 and 1/4
+        // by ~1% once the O rescale left the S -> P path).
         const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
         const float2 nm2 = make_float2(-m_used, -m_used);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -701,7 +702,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
             const float2 a = __ffma2_rn(make_float2(s[32 * c + 2 * x], s[32 * c + 2 * x + 1]), sc2, nm2);
-            const float2 pp = ((x & 7) == 7) ? exp2_poly2(a) : make_float2(ptx::ex2(a.x), ptx::ex2(a.y));
+            const float2 pp = (x == 15) ? exp2_poly2(a) : make_float2(ptx::ex2(a.x), ptx::ex2(a.y));
             acc[x & 3] = __fadd2_rn(acc[x & 3], pp);
             __nv_bfloat162 h2 = __floats2bfloat162_rn(pp.x, pp.y);
             pk[x] = *reinterpret_cast<uint32_t*>(&h2);
