@@ -169,13 +169,25 @@ const char* lite_status_string(int status);
  *                          the waits that depend on it run out their limit (no fault, no hang).
  *  LITE_OPT_MAX_CTAS       cap on the persistent grid size (0 = one CTA per SM).
  *  LITE_OPT_SCHEDULE       1 (default) = lite_attn_fwd* hand out their work items (pairs of
- *                          consecutive query tiles of one head) longest first, heads kept
- *                          together, as lite_schedule orders query tiles; 0 = in their natural
- *                          (b, h, pair) order, for measuring what the schedule buys. Results are
- *                          identical either way.
+ *                          query tiles of one head, see LITE_OPT_PAIR_STRIDE) longest first, heads
+ *                          kept together, as lite_schedule orders query tiles; 0 = in their
+ *                          natural (b, h, pair) order, for measuring what the schedule buys.
+ *                          Results are identical either way.
+ *  LITE_OPT_PAIR_STRIDE    which query tiles share a CTA (and each key tile that is live for both).
+ *                          0 (default) = chosen per call from mask_in: the stride s in [1, 64] whose
+ *                          pairs (tile r with tile r + s inside each block of 2s tiles) share the
+ *                          most live key tiles, the smaller on ties (1 = tiles 2k and 2k+1; without
+ *                          mask_in, and for lite_attn_fwd_list, 1). k >= 1 = that stride. Results
+ *                          are identical for every stride: each query tile walks its own list.
  * Returns LITE_ERR_INVALID_ARG for an unknown option or out-of-range value.
  */
-enum { LITE_OPT_WAIT_LIMIT_NS = 1, LITE_OPT_DEBUG_STALL = 2, LITE_OPT_MAX_CTAS = 3, LITE_OPT_SCHEDULE = 4 };
+enum {
+  LITE_OPT_WAIT_LIMIT_NS = 1,
+  LITE_OPT_DEBUG_STALL = 2,
+  LITE_OPT_MAX_CTAS = 3,
+  LITE_OPT_SCHEDULE = 4,
+  LITE_OPT_PAIR_STRIDE = 5
+};
 int lite_set_option(int option, long long value);
 
 /*
@@ -222,7 +234,7 @@ int lite_scratch_pool_bytes(long long* reserved);
  * by this one; lite_scratch_pool_bytes reports whether it exists).
  *
  *  - Limit: the layer's scratch must fit in 8 MiB. With R = B*H*T and T = ceil(N / tile) it is
- *    up256(2*R*T) + 2*up256(4*R) + 256 bytes (up256 rounds up to a multiple of 256), about
+ *    up256(2*R*T) + 2*up256(4*R) + 512 bytes (up256 rounds up to a multiple of 256), about
  *    R*(2T + 8). The 480p layer (B=1, H=40, N=32760, d=128: 5.3 MB) fits; the 720p layer
  *    (N=75600: 28 MB) does not. Layers that do not fit return LITE_ERR_SCRATCH_LIMIT before any
  *    work is enqueued.

@@ -1,7 +1,8 @@
 // attn_kernel.cuh -- persistent block-sparse attention forward for sm_100a (tcgen05 + TMEM + TMA).
 //
-// One CTA per SM walks a list of work items; an item is a pair of consecutive query tiles (2i,
-// 2i+1) of one (b, h). For each query tile it computes only the live key tiles of that tile
+// One CTA per SM walks a list of work items; an item is a pair of query tiles of one (b, h): tile r
+// and tile r + s of each block of 2s tiles, with the pairing stride s chosen per call as the one
+// whose pairs share the most live key tiles (s = 28 on 720p-like layers, one latent frame apart). For each query tile it computes only the live key tiles of that tile
 // (LiteAttention README, "Full-Stage Elimination": a skipped tile costs no K/V load, no QK^T, no
 // softmax, no PV), from the highest key-tile index down (README, must_do_list: "we iterate in
 // reverse order inside of the kernel"). The two query tiles share K/V: the CTA walks the union of
@@ -63,8 +64,10 @@ struct AttnParams {
   int B, H;
   int Nq, Nk;               // query / key tokens (equal for self attention)
   int Tq, Tk, W;            // query tiles, key tiles, mask words per query tile (ceil(Tk / 32))
-  int Pq;                   // query-tile pairs per (b, h): ceil(Tq / 2)
+  int Pq;                   // work items (query-tile pairs) per (b, h): ceil(Tq / 2)
   int n_items;              // B * H * Pq
+  const int* pair_stride_ptr;  // pairing stride chosen on the device for this call (null: pair_stride)
+  int pair_stride;             // pairing stride when pair_stride_ptr is null (1: tiles 2k and 2k+1)
   float scale_log2;         // softmax scale * log2(e)
   float tau_log2;           // QK-Skip threshold * log2(e)
   int skip_test;            // 1: run the QK-Skip vote and record flags
@@ -142,11 +145,28 @@ struct AttnCfg {
 // A work item as the producer hands it to the softmax warpgroups: the pair's query tiles, their
 // live counts and their first two list entries.
 struct PairInfo {
-  int row0;      // (b*H + h)*Tq + 2*qp, the first query tile's row; -1 marks the end of the work
-  int n[2];      // live key tiles of query tiles 2qp and 2qp+1 (0 when the second does not exist)
-  int b, h, qp;
+  int row0;      // (b*H + h)*Tq: the head's first query-tile row; -1 marks the end of the work
+  int n[2];      // live key tiles of the pair's two query tiles (0 when the second does not exist)
+  int qt[2];     // the two query tiles (qt[1] = Tq when the item has one query tile)
+  int b, h;
   int e[2][2];   // entries 0 and 1 of each query tile's list
 };
+
+// The query tiles of work item k (0 <= k < ceil(T/2)) of a head under pairing stride s: inside each
+// block of 2s tiles, tile r pairs with tile r + s (r < s); the tiles after the last full block pair
+// as (t, t+1). Stride 1 pairs 2k with 2k+1. b = -1 when the item has one tile (odd T).
+__device__ __forceinline__ void pair_tiles(int k, int T, int s, int& a, int& b) {
+  const int full = (T / (2 * s)) * (2 * s);
+  if (2 * k < full) {
+    const int blk = k / s;
+    a = blk * 2 * s + (k - blk * s);
+    b = a + s;
+  } else {
+    a = full + 2 * (k - full / 2);
+    b = a + 1;
+  }
+  if (b >= T) b = -1;
+}
 
 // Per union tile, what the producer tells the MMA thread (one 32-bit word in a 4-slot ring).
 constexpr uint32_t kLive0 = 1u, kLive1 = 2u;        // live for query tile 0 / 1
@@ -262,7 +282,7 @@ __device__ __forceinline__ int key_entry(const AttnParams& p, int row, int idx) 
 
 // Work item `item` (in hand-out order) decoded: the pair's rows, live counts and first entries.
 // Returns false (and a pair with no live tiles) when the work order or a live count is out of range.
-__device__ __forceinline__ bool decode_pair(const AttnParams& p, int item, PairInfo& it) {
+__device__ __forceinline__ bool decode_pair(const AttnParams& p, int item, int stride, PairInfo& it) {
   const int pair = p.order ? p.order[item] : item;
   if (pair < 0 || pair >= p.n_items) {
     it.row0 = 0;
@@ -270,15 +290,19 @@ __device__ __forceinline__ bool decode_pair(const AttnParams& p, int item, PairI
     return false;
   }
   const int bh = pair / p.Pq;
-  it.qp = pair - bh * p.Pq;
+  const int k = pair - bh * p.Pq;
   it.b = bh / p.H;
   it.h = bh - it.b * p.H;
-  it.row0 = bh * p.Tq + 2 * it.qp;
+  it.row0 = bh * p.Tq;
+  int a, b;
+  pair_tiles(k, p.Tq, stride, a, b);
+  it.qt[0] = a;
+  it.qt[1] = b >= 0 ? b : p.Tq;
   bool ok = true;
 #pragma unroll
   for (int g = 0; g < 2; ++g) {
-    const bool exists = 2 * it.qp + g < p.Tq;
-    int n = !exists ? 0 : (p.counts ? p.counts[it.row0 + g] : p.Tk);
+    const bool exists = it.qt[g] < p.Tq;
+    int n = !exists ? 0 : (p.counts ? p.counts[it.row0 + it.qt[g]] : p.Tk);
     if (n < 0 || n > p.Tk) {
       ok = false;
       n = 0;
@@ -288,8 +312,8 @@ __device__ __forceinline__ bool decode_pair(const AttnParams& p, int item, PairI
   if (!ok) it.n[0] = it.n[1] = 0;
 #pragma unroll
   for (int g = 0; g < 2; ++g) {
-    it.e[g][0] = it.n[g] > 0 ? key_entry(p, it.row0 + g, 0) : 0;
-    it.e[g][1] = it.n[g] > 1 ? key_entry(p, it.row0 + g, 1) : 0;
+    it.e[g][0] = it.n[g] > 0 ? key_entry(p, it.row0 + it.qt[g], 0) : 0;
+    it.e[g][1] = it.n[g] > 1 ? key_entry(p, it.row0 + it.qt[g], 1) : 0;
   }
   return ok;
 }
@@ -398,6 +422,7 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       uint32_t u = 0, items = 0, qn = 0, live_pairs = 0;
       bool ok = true;
+      const int stride = p.pair_stride_ptr ? *p.pair_stride_ptr : p.pair_stride;
       // last armed phase of each full barrier, so that every issued load can be drained at exit
       bool q_armed = false, kv_armed[2] = {false, false};
       uint32_t q_par = 0, kv_par[2] = {0, 0};
@@ -434,7 +459,7 @@ __global__ void __launch_bounds__(320, 1)
         PairInfo it{};
         it.row0 = -1;
         bool good = true;
-        if (item >= 0) good = decode_pair(p, item, it);
+        if (item >= 0) good = stride >= 1 && decode_pair(p, item, stride, it);
         if (!good) it.row0 = -1;  // the softmax groups stop as at the end of the work
         ctl->info[slot] = it;
         ptx::mbar_arrive(BAR(item_full[slot]));
@@ -460,13 +485,13 @@ __global__ void __launch_bounds__(320, 1)
         ptx::mbar_arrive_expect_tx(BAR(q_full), (it.n[0] > 0 ? C::Q_TX : 0u) + (it.n[1] > 0 ? C::Q_TX : 0u));
         for (int g = 0; g < 2; ++g)
           if (it.n[g] > 0)
-            ptx::tma_load_5d(sQ + g * C::Q_BYTES + g * C::ROW1 * 128, &tmQ, BAR(q_full), 0, (2 * it.qp + g) * C::BQ, 0,
-                             it.h, it.b);
+            ptx::tma_load_5d(sQ + g * C::Q_BYTES + g * C::ROW1 * 128, &tmQ, BAR(q_full), 0, it.qt[g] * C::BQ, 0, it.h,
+                             it.b);
         q_armed = true;
         q_par = qn & 1;
         // the union of the two descending lists, highest key tile first
-        ListCursor c0{it.row0, it.n[0], 0, it.e[0][0], it.e[0][1], p.Tk};
-        ListCursor c1{it.row0 + 1, it.n[1], 0, it.e[1][0], it.e[1][1], p.Tk};
+        ListCursor c0{it.row0 + it.qt[0], it.n[0], 0, it.e[0][0], it.e[0][1], p.Tk};
+        ListCursor c1{it.row0 + it.qt[1], it.n[1], 0, it.e[1][0], it.e[1][1], p.Tk};
         const uint32_t item_bits = ((qn & 1) ? kItemOdd : 0u) | (qn >= 1 ? kItemAfterFirst : 0u);
         uint32_t f = kItemFirst;
         while (ok) {
@@ -597,7 +622,7 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------------------- softmax warpgroups
-    const int grp = (warp - 2) >> 2;                // query tile 2qp + grp of each pair
+    const int grp = (warp - 2) >> 2;                // query tile qt[grp] of each pair
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;              // TMEM lane = row inside the tile slot
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
@@ -616,9 +641,9 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) ptx::mbar_arrive(BAR(item_empty[slot]));
       ++items;
       if (!ptx::named_bar_and(gbar, 128, ok) || it.row0 < 0) break;
-      const int qi = 2 * it.qp + grp;
+      const int qi = it.qt[grp];  // Tq when the item has no second query tile
       const int n = it.n[grp];
-      const int row = it.row0 + grp;
+      const int row = it.row0 + qi;
       const int rq = r - grp * C::ROW1;  // row inside the query tile
       const int n_row = qi * C::BQ + rq;
       const bool valid_row = qi < p.Tq && rq >= 0 && rq < C::BQ && n_row < p.Nq;

@@ -32,6 +32,7 @@ struct Options {
   int debug_stall = 0;
   int max_ctas = 0;
   int schedule = 1;
+  int pair_stride = 0;  // 0: chosen per call from the mask; k >= 1: query tiles r and r + k paired
 };
 Options g_opt;
 unsigned long long* g_cta_times = nullptr;
@@ -203,6 +204,7 @@ lite::AttnParams base_params(void* o, float* lse, int B, int H, int Nq, int Nk, 
   p.W = (p.Tk + 31) / 32;
   p.Pq = (p.Tq + 1) / 2;
   p.n_items = B * H * p.Pq;  // work items: pairs of query tiles
+  p.pair_stride = 1;
   p.scale_log2 = resolve_scale(scale, d) * 1.4426950408889634f;
   p.tau_log2 = -INFINITY;
   p.status = dc->status;
@@ -247,10 +249,48 @@ int validate_fwd(const FwdArgs& a) {
   return LITE_OK;
 }
 
-// Scratch layout: live lists [rows, Tk] int16 | counts [rows] | order [rows] | work counter.
+// Scratch layout: live lists [rows, Tk] int16 | counts [rows] | order [rows] | a 512-byte tail with
+// the work counter (+0), the chosen pairing stride (+4) and the stride scores (+256, 64 x uint32).
+constexpr size_t kTailBytes = 512;
 struct FwdScratch {
   size_t list_b, cnt_b, total;
 };
+struct Tail {
+  int32_t* counter;
+  int32_t* stride;
+  uint32_t* scores;
+};
+Tail tail_at(char* t) {
+  return Tail{reinterpret_cast<int32_t*>(t), reinterpret_cast<int32_t*>(t + 4), reinterpret_cast<uint32_t*>(t + 256)};
+}
+
+// Enqueues the pairing-stride choice (when the option leaves it to the mask) and the pair schedule;
+// fills the attention parameters' work order, counter and stride.
+int enqueue_pairs(const FwdArgs& a, const uint32_t* mask_in, const int32_t* counts, int32_t* order, char* tail,
+                  lite::AttnParams& p, cudaStream_t s) {
+  const Tail t = tail_at(tail);
+  const int Tq = p.Tq, BH = a.B * a.H;
+  const int n_cand = std::max(1, std::min(lite::kMaxPairStride, Tq / 2));
+  const bool scored = g_opt.pair_stride == 0 && mask_in != nullptr && n_cand > 1;
+  if (scored) {
+    const int chunks = std::max(1, std::min(8, BH));
+    lite::lite_stride_score_kernel<<<dim3(n_cand, chunks), 256, 0, s>>>(mask_in, t.scores, BH, Tq, p.Tk, p.W);
+    if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
+  }
+  if (g_opt.schedule) {
+    const size_t sm = size_t(BH + p.Pq) * sizeof(int32_t);
+    lite::lite_schedule_kernel<2><<<BH, 512, sm, s>>>(counts, order, BH, Tq, scored ? t.scores : nullptr, n_cand,
+                                                      g_opt.pair_stride, t.stride);
+    if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
+    p.pair_stride_ptr = t.stride;  // written by the schedule kernel
+  } else {
+    p.pair_stride_ptr = nullptr;
+    p.pair_stride = g_opt.pair_stride >= 1 ? g_opt.pair_stride : 1;
+  }
+  p.order = g_opt.schedule ? order : nullptr;  // null: pairs in their natural order
+  p.work_counter = t.counter;
+  return LITE_OK;
+}
 
 FwdScratch fwd_scratch(const FwdArgs& a) {
   const int t = tile_for(a.d);
@@ -259,7 +299,7 @@ FwdScratch fwd_scratch(const FwdArgs& a) {
   FwdScratch f;
   f.list_b = align256(rows * Tk * sizeof(int16_t));
   f.cnt_b = align256(rows * sizeof(int32_t));
-  f.total = f.list_b + 2 * f.cnt_b + 256;
+  f.total = f.list_b + 2 * f.cnt_b + kTailBytes;
   return f;
 }
 
@@ -296,10 +336,10 @@ int enqueue_fwd(DeviceCache* dc, const FwdArgs& a, const lite::RangeBits* ranges
   int16_t* list = reinterpret_cast<int16_t*>(base);
   int32_t* counts = reinterpret_cast<int32_t*>(base + f.list_b);
   int32_t* order = reinterpret_cast<int32_t*>(base + f.list_b + f.cnt_b);
-  int32_t* counter = reinterpret_cast<int32_t*>(base + f.list_b + 2 * f.cnt_b);
+  char* tail = base + f.list_b + 2 * f.cnt_b;
 
-  // the work counter must start at zero (fixed scratch keeps the previous call's value)
-  if (cudaMemsetAsync(counter, 0, sizeof(int32_t), s) != cudaSuccess) return LITE_ERR_CUDA;
+  // the work counter and the stride scores must start at zero (fixed scratch keeps the last call's)
+  if (cudaMemsetAsync(tail, 0, kTailBytes, s) != cudaSuccess) return LITE_ERR_CUDA;
   const int cblocks = (rows + 7) / 8;
   if (ranges)
     lite::lite_compact_kernel<true><<<cblocks, 256, 0, s>>>(a.mask_in, a.mask_out, list, counts, rows, Tk, W, *ranges);
@@ -307,16 +347,11 @@ int enqueue_fwd(DeviceCache* dc, const FwdArgs& a, const lite::RangeBits* ranges
     lite::lite_compact_kernel<false><<<cblocks, 256, 0, s>>>(a.mask_in, a.mask_out, list, counts, rows, Tk, W,
                                                              lite::RangeBits{});
   if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
-  if (g_opt.schedule) {
-    const size_t sm = size_t(a.B * a.H + p.Pq) * sizeof(int32_t);
-    lite::lite_schedule_kernel<2><<<a.B * a.H, 512, sm, s>>>(counts, order, a.B * a.H, Tq);
-    if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
-  }
+  int st = enqueue_pairs(a, a.mask_in, counts, order, tail, p, s);
+  if (st) return st;
   p.mask_out = a.mask_out;
   p.list = list;
   p.counts = counts;
-  p.order = g_opt.schedule ? order : nullptr;  // null: pairs in their natural order
-  p.work_counter = counter;
   p.tau_log2 = a.tau * 1.4426950408889634f;
   p.skip_test = (a.mask_out != nullptr && a.tau > -INFINITY) ? 1 : 0;
   return run_attention(dc, a.d, a.q, a.k, a.v, p, s);
@@ -327,26 +362,22 @@ int enqueue_fwd(DeviceCache* dc, const FwdArgs& a, const lite::RangeBits* ranges
 size_t list_scratch_bytes(const FwdArgs& a) {
   const int t = tile_for(a.d);
   const size_t rows = size_t(a.B) * a.H * ((a.Nq + t - 1) / t);
-  return align256(rows * sizeof(int32_t)) + 256;
+  return align256(rows * sizeof(int32_t)) + kTailBytes;
 }
 
 int enqueue_list(DeviceCache* dc, const FwdArgs& a, const int16_t* list, const int32_t* counts, char* base,
                  cudaStream_t s) {
   lite::AttnParams p = base_params(a.o, a.lse, a.B, a.H, a.Nq, a.Nk, a.d, a.scale, dc);
-  const int Tq = p.Tq, rows = a.B * a.H * Tq;
+  const int rows = a.B * a.H * p.Tq;
   int32_t* order = reinterpret_cast<int32_t*>(base);
-  int32_t* counter = reinterpret_cast<int32_t*>(base + align256(size_t(rows) * sizeof(int32_t)));
-  if (cudaMemsetAsync(counter, 0, sizeof(int32_t), s) != cudaSuccess) return LITE_ERR_CUDA;
-  if (g_opt.schedule) {
-    const size_t sm = size_t(a.B * a.H + p.Pq) * sizeof(int32_t);
-    lite::lite_schedule_kernel<2><<<a.B * a.H, 512, sm, s>>>(counts, order, a.B * a.H, Tq);
-    if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
-  }
+  char* tail = base + align256(size_t(rows) * sizeof(int32_t));
+  if (cudaMemsetAsync(tail, 0, kTailBytes, s) != cudaSuccess) return LITE_ERR_CUDA;
+  // no mask here: the pairing stride is the option's, or 1
+  int st = enqueue_pairs(a, nullptr, counts, order, tail, p, s);
+  if (st) return st;
   p.mask_out = a.mask_out;
   p.list = list;
   p.counts = counts;
-  p.order = g_opt.schedule ? order : nullptr;
-  p.work_counter = counter;
   p.tau_log2 = a.tau * 1.4426950408889634f;
   p.skip_test = (a.mask_out != nullptr && a.tau > -INFINITY) ? 1 : 0;
   return run_attention(dc, a.d, a.q, a.k, a.v, p, s);
@@ -409,6 +440,10 @@ int lite_set_option(int option, long long value) {
     case LITE_OPT_MAX_CTAS:
       if (value < 0 || value > 1000000) return LITE_ERR_INVALID_ARG;
       g_opt.max_ctas = static_cast<int>(value);
+      return LITE_OK;
+    case LITE_OPT_PAIR_STRIDE:
+      if (value < 0 || value > kMaxT) return LITE_ERR_INVALID_ARG;
+      g_opt.pair_stride = static_cast<int>(value);
       return LITE_OK;
     default:
       return LITE_ERR_INVALID_ARG;

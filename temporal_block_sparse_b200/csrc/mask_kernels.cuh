@@ -7,10 +7,16 @@
 //    which is where the attention kernel later ORs new flags. With must-do / must-skip ranges the
 //    live set is (not masked or must-do) and not (must-skip and not must-do); must-do entries are
 //    tagged so that the attention kernel never flags them. The copied mask is mask_in unchanged.
+//  * lite_stride_score_kernel: for each candidate pairing stride s, the number of live key tiles
+//    the attention kernel's query-tile pairs would share (summed over heads). A key tile live for
+//    both query tiles of a pair is loaded once and computed for both with their softmaxes
+//    overlapping; one live for only one of them runs alone. Pairing the tiles that share the most
+//    live key tiles therefore cuts such lone tiles: on the 720p-like layers the best stride is 28,
+//    the tiles one latent frame apart (3600 tokens per frame / 128).
 //  * lite_schedule_kernel: one CTA per head. Ranks the head among all heads by total live work,
 //    then places each of its work items (query tiles, or pairs of query tiles) by (live count
 //    desc, index asc) with an O(T^2) rank count in shared memory -- deterministic, no atomics on
-//    the output.
+//    the output. For pairs it first picks the stride with the best score (ties: the smaller).
 #pragma once
 
 #include <stdint.h>
@@ -137,18 +143,76 @@ __global__ void __launch_bounds__(256) lite_ranges_kernel(const uint32_t* __rest
   if (lane == 0) nruns[row] = count / 2;
 }
 
+constexpr int kMaxPairStride = 64;
+
+// Candidate stride s = blockIdx.x + 1; blockIdx.y splits the heads. scores[s-1] (zeroed before the
+// launch) += live key tiles shared by the pairs of stride s, over this block's heads. Every mask row
+// is read whole (bits >= Tk of the last word cleared).
+__global__ void __launch_bounds__(256) lite_stride_score_kernel(const uint32_t* __restrict__ mask,
+                                                               uint32_t* __restrict__ scores, int BH, int T, int Tk,
+                                                               int W) {
+  const int s = blockIdx.x + 1;
+  const int P = (T + 1) / 2;  // T: query tiles per head; Tk: key tiles (bits per row)
+  const uint32_t tail_mask = (Tk & 31) ? ((1u << (Tk & 31)) - 1u) : 0xffffffffu;
+  const long long items = static_cast<long long>(BH) * P;
+  const long long per = (items + gridDim.y - 1) / gridDim.y;
+  const long long lo = per * blockIdx.y, hi = min(items, lo + per);
+  uint32_t acc = 0;
+  for (long long x = lo + threadIdx.x; x < hi; x += blockDim.x) {
+    const int bh = int(x / P);
+    const int k = int(x - static_cast<long long>(bh) * P);
+    int a, b;
+    pair_tiles(k, T, s, a, b);
+    if (b < 0) continue;
+    const uint32_t* ra = mask + (size_t(bh) * T + a) * W;
+    const uint32_t* rb = mask + (size_t(bh) * T + b) * W;
+    for (int w = 0; w < W; ++w) {
+      const uint32_t valid = (w == W - 1) ? tail_mask : 0xffffffffu;
+      acc += __popc(~__ldg(ra + w) & ~__ldg(rb + w) & valid);
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  __shared__ uint32_t part[8];
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t t = 0;
+    for (int i = 0; i < int(blockDim.x >> 5); ++i) t += part[i];
+    if (t) atomicAdd(scores + (s - 1), t);
+  }
+}
+
+// The pairing stride for G = 2: fixed_stride if >= 1, else the candidate with the highest score
+// (the smaller stride on ties), 1 without scores.
+__device__ __forceinline__ int pick_stride(const uint32_t* scores, int n_cand, int fixed_stride) {
+  if (fixed_stride >= 1) return fixed_stride;
+  if (!scores) return 1;
+  int best = 1;
+  uint32_t top = scores[0];
+  for (int x = 1; x < n_cand; ++x)
+    if (scores[x] > top) {
+      top = scores[x];
+      best = x + 1;
+    }
+  return best;
+}
+
 // smem: totals[BH] ints, then counts of this head [T] ints
-// G = 1 orders the query tiles of every head; G = 2 orders pairs of consecutive query tiles
-// (2i, 2i+1), the work items of the attention kernel, by their combined live count. Output entries
-// are head * ceil(T/G) + item.
+// G = 1 orders the query tiles of every head; G = 2 orders pairs of query tiles (pair_tiles with the
+// picked stride, which CTA 0 also writes to *stride_out), the work items of the attention kernel, by
+// their combined live count. Output entries are head * ceil(T/G) + item.
 template <int G>
 __global__ void __launch_bounds__(512) lite_schedule_kernel(const int32_t* __restrict__ counts,
-                                                           int32_t* __restrict__ order, int BH, int T) {
+                                                           int32_t* __restrict__ order, int BH, int T,
+                                                           const uint32_t* scores = nullptr, int n_cand = 0,
+                                                           int fixed_stride = 0, int* stride_out = nullptr) {
   extern __shared__ int32_t sh[];
   const int P = (T + G - 1) / G;  // items per head
   int32_t* totals = sh;
   int32_t* mine = sh + BH;
   const int g = blockIdx.x;
+  const int stride = G == 2 ? pick_stride(scores, n_cand, fixed_stride) : 1;
+  if (G == 2 && g == 0 && threadIdx.x == 0 && stride_out) *stride_out = stride;
   for (int x = threadIdx.x; x < BH; x += blockDim.x) totals[x] = 0;
   __syncthreads();
   // per-head totals (every CTA computes all of them; B*H*T ints, served from L2)
@@ -157,10 +221,14 @@ __global__ void __launch_bounds__(512) lite_schedule_kernel(const int32_t* __res
     if (v) atomicAdd(&totals[x / T], v);
   }
   for (int x = threadIdx.x; x < P; x += blockDim.x) {
-    int c = 0;
-#pragma unroll
-    for (int k = 0; k < G; ++k)
-      if (G * x + k < T) c += __ldg(counts + size_t(g) * T + G * x + k);
+    int c;
+    if constexpr (G == 2) {
+      int a, b;
+      pair_tiles(x, T, stride, a, b);
+      c = __ldg(counts + size_t(g) * T + a) + (b >= 0 ? __ldg(counts + size_t(g) * T + b) : 0);
+    } else {
+      c = __ldg(counts + size_t(g) * T + x);
+    }
     mine[x] = c;
   }
   __syncthreads();

@@ -417,6 +417,7 @@ def lite_mask_to_ranges(mask: Optional[torch.Tensor], B: int, H: int, N: int, d:
 
 
 LITE_OPT_SCHEDULE = 4
+LITE_OPT_PAIR_STRIDE = 5
 
 
 def lite_set_cta_timing(buf: Optional[torch.Tensor]):

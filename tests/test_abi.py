@@ -235,3 +235,7 @@ def test_cta_timing_and_schedule_option_checks():
     assert lib.lite_set_option(la.LITE_OPT_SCHEDULE, 2) == la.LITE_ERR_INVALID_ARG
     assert lib.lite_set_option(la.LITE_OPT_SCHEDULE, 0) == la.LITE_OK
     assert lib.lite_set_option(la.LITE_OPT_SCHEDULE, 1) == la.LITE_OK
+    assert lib.lite_set_option(la.LITE_OPT_PAIR_STRIDE, -1) == la.LITE_ERR_INVALID_ARG
+    assert lib.lite_set_option(la.LITE_OPT_PAIR_STRIDE, 4097) == la.LITE_ERR_INVALID_ARG
+    assert lib.lite_set_option(la.LITE_OPT_PAIR_STRIDE, 28) == la.LITE_OK
+    assert lib.lite_set_option(la.LITE_OPT_PAIR_STRIDE, 0) == la.LITE_OK

@@ -1,6 +1,8 @@
-"""The longest-first work order changes only which CTA processes which query tile (needs a B200).
+"""The work order and the pairing of query tiles change only which CTA processes which query tile
+(needs a B200).
 
-Results (o, lse, mask) are bit-identical with the schedule on and off; the per-CTA timing hook
+Results (o, lse, mask) are bit-identical with the schedule on and off and for every pairing stride
+(each query tile walks its own Skip-List whatever tile it shares a CTA with); the per-CTA timing hook
 accounts for every live tile exactly once.
 """
 
@@ -19,6 +21,7 @@ def _clean_state():
     la.load()
     yield
     la.lite_set_option(la.LITE_OPT_SCHEDULE, 1)
+    la.lite_set_option(la.LITE_OPT_PAIR_STRIDE, 0)
     la.lite_set_cta_timing(None)
     assert la.lite_get_device_status() == 0
 
@@ -63,7 +66,47 @@ def test_cta_timing_counts_every_live_tile():
     la.lite_set_cta_timing(None)
     rec = buf.cpu().numpy()
     used = rec[:, 1] > 0
-    # the kernel's work items are pairs of query tiles (2i, 2i+1) of one head
+    # the kernel's work items are pairs of query tiles of one head
     assert used.sum() == min(sms, B * H * ((T + 1) // 2))
     assert (rec[used, 1] >= rec[used, 0]).all()
     assert int(rec[used, 2].sum()) == live
+
+
+def _run_with(q, k, v, m_in, tau, **opts):
+    for name, val in opts.items():
+        la.lite_set_option(getattr(la, name), val)
+    m_out = torch.empty_like(m_in)
+    o, lse = la.lite_attn_fwd(q, k, v, m_in, m_out, tau=tau)
+    torch.cuda.synchronize()
+    assert la.lite_get_device_status() == 0
+    return o.clone(), lse.clone(), m_out.clone()
+
+
+@pytest.mark.parametrize("layer", ["small", "480p"])
+def test_pairing_stride_gives_identical_results(layer):
+    """Fixed strides (1 = tiles 2k and 2k+1, several others, and strides larger than half the
+    query tiles) and the stride picked from the mask give the same bits, with the schedule on and
+    off. The 480p case runs six steps of its trajectory first, so the mask is the grown, uneven one
+    where the picked stride differs from 1."""
+    if layer == "small":
+        (q, k, v), m_in = _masked_step(63)
+        tau = -2.0
+    else:
+        w = wl.WORKLOADS["480p"]
+        tr = wl.Trajectory(w, device="cuda")
+        B, N, H, d = w.B, w.N, w.H, w.d
+        m_in = la.new_mask(B, H, N, d)
+        m_out = torch.empty_like(m_in)
+        for t in range(6):
+            q, k, v = tr.current()
+            la.lite_attn_fwd(q, k, v, m_in, m_out, tau=w.tau(t))
+            m_in, m_out = m_out, m_in
+            tr.advance()
+        q, k, v = tr.current()
+        tau = w.tau(6)
+    ref = _run_with(q, k, v, m_in, tau, LITE_OPT_PAIR_STRIDE=1, LITE_OPT_SCHEDULE=1)
+    for stride in (0, 2, 3, 12, 28, 64, 4096):
+        for sched in (1, 0):
+            got = _run_with(q, k, v, m_in, tau, LITE_OPT_PAIR_STRIDE=stride, LITE_OPT_SCHEDULE=sched)
+            for a, b in zip(ref, got):
+                assert torch.equal(a, b), (stride, sched)
