@@ -63,8 +63,9 @@ struct AttnParams {
   int* status;              // device status word
   int B, H;
   int Nq, Nk;               // query / key tokens (equal for self attention)
-  int Tq, Tk, W;            // query tiles, key tiles, mask words per query tile (ceil(Tk / 32))
-  int Pq;                   // work items (query-tile pairs) per (b, h): ceil(Tq / 2)
+  int Tq, Tk, W;            // query tiles (mask rows), key tiles, mask words per row (ceil(Tk / 32))
+  int Tkq;                  // kernel query tiles per (b, h): ceil(Tq / MR)
+  int Pq;                   // work items (kernel query-tile pairs) per (b, h): ceil(Tkq / 2)
   int n_items;              // B * H * Pq
   const int* pair_stride_ptr;  // pairing stride chosen on the device for this call (null: pair_stride)
   int pair_stride;             // pairing stride when pair_stride_ptr is null (1: tiles 2k and 2k+1)
@@ -96,11 +97,14 @@ struct AttnParams {
 template <int D, int BN>
 struct AttnCfg {
   static constexpr int BM = 128;                 // MMA M = TMEM lanes = query rows of a tile slot
-  static constexpr int BQ = BN;                  // valid query rows per query tile
-  // Rows of query tile g sit at TMEM lanes / smem rows [g*ROW1, g*ROW1 + BQ). With 64-row tiles
-  // (d = 64) the second tile takes the upper half, so the useful softmax warps of the two groups
-  // fall on different scheduler partitions.
-  static constexpr int ROW1 = BM - BQ;
+  // A kernel query tile has 128 rows. With 64-row Skip-Mask tiles (d = 64) it stacks MR = 2
+  // consecutive mask rows (query tiles of the mask): rows 0-63 are mask row 2m, rows 64-127 mask
+  // row 2m+1, so every MMA row is a query row. Each half keeps its own Skip-List, running max and
+  // QK-Skip vote; a key tile live for only one half computes the other half's rows too and gives
+  // them P = 0.
+  static constexpr int MR = BM / BN;             // mask rows per kernel query tile: 1 (d=128), 2 (d=64)
+  static constexpr int BQ = BM;                  // query rows per kernel query tile
+  static constexpr int ROW1 = BM - BQ;           // 0: both query-tile slots are full
   static constexpr int THREADS = 320;            // producer warp, MMA warp, 2 softmax warpgroups
   static constexpr int NCHUNK = D / 64;          // 128-byte swizzle atoms along d
   static constexpr int Q_CHUNK = BM * 128;       // bytes between d-chunks of a Q tile in smem
@@ -145,11 +149,14 @@ struct AttnCfg {
 // A work item as the producer hands it to the softmax warpgroups: the pair's query tiles, their
 // live counts and their first two list entries.
 struct PairInfo {
-  int row0;      // (b*H + h)*Tq: the head's first query-tile row; -1 marks the end of the work
+  int row0;      // (b*H + h)*Tq: the head's first mask row; -1 marks the end of the work
   int n[2];      // live key tiles of the pair's two query tiles (0 when the second does not exist)
-  int qt[2];     // the two query tiles (qt[1] = Tq when the item has one query tile)
+  int qt[2];     // the two kernel query tiles (qt[1] = Tkq when the item has one)
   int b, h;
   int e[2][2];   // entries 0 and 1 of each query tile's list
+  // second mask row of each kernel query tile (MR = 2 only): live count and entries 0 and 1
+  int n2[2];
+  int e2[2][2];
 };
 
 // The query tiles of work item k (0 <= k < ceil(T/2)) of a head under pairing stride s: inside each
@@ -282,11 +289,13 @@ __device__ __forceinline__ int key_entry(const AttnParams& p, int row, int idx) 
 
 // Work item `item` (in hand-out order) decoded: the pair's rows, live counts and first entries.
 // Returns false (and a pair with no live tiles) when the work order or a live count is out of range.
+template <int MR>
 __device__ __forceinline__ bool decode_pair(const AttnParams& p, int item, int stride, PairInfo& it) {
   const int pair = p.order ? p.order[item] : item;
   if (pair < 0 || pair >= p.n_items) {
     it.row0 = 0;
     it.n[0] = it.n[1] = 0;
+    it.n2[0] = it.n2[1] = 0;
     return false;
   }
   const int bh = pair / p.Pq;
@@ -295,26 +304,43 @@ __device__ __forceinline__ bool decode_pair(const AttnParams& p, int item, int s
   it.h = bh - it.b * p.H;
   it.row0 = bh * p.Tq;
   int a, b;
-  pair_tiles(k, p.Tq, stride, a, b);
+  pair_tiles(k, p.Tkq, stride, a, b);
   it.qt[0] = a;
-  it.qt[1] = b >= 0 ? b : p.Tq;
+  it.qt[1] = b >= 0 ? b : p.Tkq;
   bool ok = true;
+  int n[2][MR];
 #pragma unroll
-  for (int g = 0; g < 2; ++g) {
-    const bool exists = it.qt[g] < p.Tq;
-    int n = !exists ? 0 : (p.counts ? p.counts[it.row0 + it.qt[g]] : p.Tk);
-    if (n < 0 || n > p.Tk) {
-      ok = false;
-      n = 0;
+  for (int g = 0; g < 2; ++g)
+#pragma unroll
+    for (int hf = 0; hf < MR; ++hf) {
+      const int mrow = it.qt[g] * MR + hf;
+      const bool exists = it.qt[g] < p.Tkq && mrow < p.Tq;
+      int c = !exists ? 0 : (p.counts ? p.counts[it.row0 + mrow] : p.Tk);
+      if (c < 0 || c > p.Tk) {
+        ok = false;
+        c = 0;
+      }
+      n[g][hf] = c;
     }
-    it.n[g] = n;
-  }
-  if (!ok) it.n[0] = it.n[1] = 0;
 #pragma unroll
-  for (int g = 0; g < 2; ++g) {
-    it.e[g][0] = it.n[g] > 0 ? key_entry(p, it.row0 + it.qt[g], 0) : 0;
-    it.e[g][1] = it.n[g] > 1 ? key_entry(p, it.row0 + it.qt[g], 1) : 0;
-  }
+  for (int g = 0; g < 2; ++g)
+#pragma unroll
+    for (int hf = 0; hf < MR; ++hf) {
+      const int c = ok ? n[g][hf] : 0;
+      const int r = it.row0 + it.qt[g] * MR + hf;
+      const int e0 = c > 0 ? key_entry(p, r, 0) : 0;
+      const int e1 = c > 1 ? key_entry(p, r, 1) : 0;
+      if (hf == 0) {
+        it.n[g] = c;
+        it.e[g][0] = e0;
+        it.e[g][1] = e1;
+      } else {
+        it.n2[g] = c;
+        it.e2[g][0] = e0;
+        it.e2[g][1] = e1;
+      }
+    }
+  if constexpr (MR == 1) it.n2[0] = it.n2[1] = 0;
   return ok;
 }
 
@@ -459,7 +485,7 @@ __global__ void __launch_bounds__(320, 1)
         PairInfo it{};
         it.row0 = -1;
         bool good = true;
-        if (item >= 0) good = stride >= 1 && decode_pair(p, item, stride, it);
+        if (item >= 0) good = stride >= 1 && decode_pair<C::MR>(p, item, stride, it);
         if (!good) it.row0 = -1;  // the softmax groups stop as at the end of the work
         ctl->info[slot] = it;
         ptx::mbar_arrive(BAR(item_full[slot]));
@@ -470,7 +496,8 @@ __global__ void __launch_bounds__(320, 1)
           break;
         }
         if (item < 0) break;
-        if (it.n[0] + it.n[1] == 0) {
+        const int gn[2] = {it.n[0] + it.n2[0], it.n[1] + it.n2[1]};  // live tiles per kernel query tile
+        if (gn[0] + gn[1] == 0) {
           // An item without tiles needs no bundle. But a softmax group may still wait, in the
           // epilogue of its previous item, for the PV of that item's last union tile, which the MMA
           // thread issues with the next bundle; and before this producer hands out two more items,
@@ -482,18 +509,19 @@ __global__ void __launch_bounds__(320, 1)
         // the pair's Q tiles; q_empty is committed after the item's last QK
         if (qn >= 1) ok = wt.wait(BAR(q_empty), (qn - 1) & 1);
         if (!ok) break;
-        ptx::mbar_arrive_expect_tx(BAR(q_full), (it.n[0] > 0 ? C::Q_TX : 0u) + (it.n[1] > 0 ? C::Q_TX : 0u));
+        ptx::mbar_arrive_expect_tx(BAR(q_full), (gn[0] > 0 ? C::Q_TX : 0u) + (gn[1] > 0 ? C::Q_TX : 0u));
         for (int g = 0; g < 2; ++g)
-          if (it.n[g] > 0)
+          if (gn[g] > 0)
             ptx::tma_load_5d(sQ + g * C::Q_BYTES + g * C::ROW1 * 128, &tmQ, BAR(q_full), 0, it.qt[g] * C::BQ, 0, it.h,
                              it.b);
         q_armed = true;
         q_par = qn & 1;
+        const uint32_t item_bits = ((qn & 1) ? kItemOdd : 0u) | (qn >= 1 ? kItemAfterFirst : 0u);
+        uint32_t f = kItemFirst;
+        if constexpr (C::MR == 1) {
         // the union of the two descending lists, highest key tile first
         ListCursor c0{it.row0 + it.qt[0], it.n[0], 0, it.e[0][0], it.e[0][1], p.Tk};
         ListCursor c1{it.row0 + it.qt[1], it.n[1], 0, it.e[1][0], it.e[1][1], p.Tk};
-        const uint32_t item_bits = ((qn & 1) ? kItemOdd : 0u) | (qn >= 1 ? kItemAfterFirst : 0u);
-        uint32_t f = kItemFirst;
         while (ok) {
           const int h0 = c0.head(), h1 = c1.head();
           const int j = max(h0, h1);
@@ -513,7 +541,50 @@ __global__ void __launch_bounds__(320, 1)
           if (last) break;
           f = 0u;
         }
-        live_pairs += uint32_t(it.n[0] + it.n[1]);
+        } else {
+        // Stacked rows: kernel query tile g has two mask rows, each with its own list. The key tiles
+        // of the item are the union of the four lists; tile j is computed for kernel tile g when it
+        // is live for either of g's rows.
+        ListCursor cur[2][2] = {
+            {{it.row0 + it.qt[0] * 2, it.n[0], 0, it.e[0][0], it.e[0][1], p.Tk},
+             {it.row0 + it.qt[0] * 2 + 1, it.n2[0], 0, it.e2[0][0], it.e2[0][1], p.Tk}},
+            {{it.row0 + it.qt[1] * 2, it.n[1], 0, it.e[1][0], it.e[1][1], p.Tk},
+             {it.row0 + it.qt[1] * 2 + 1, it.n2[1], 0, it.e2[1][0], it.e2[1][1], p.Tk}}};
+        bool started[2] = {false, false};
+        while (ok) {
+          int j = -1;
+#pragma unroll
+          for (int g = 0; g < 2; ++g) j = max(j, max(cur[g][0].head(), cur[g][1].head()));
+          f |= item_bits;
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            bool live = false;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+              if (cur[g][hf].head() == j) {
+                if (!cur[g][hf].head_ok()) ok = false;  // malformed or not strictly descending
+                cur[g][hf].advance(p);
+                live = true;
+              }
+            if (live) {
+              f |= (kLive0 << g) | (started[g] ? 0u : (kFirst0 << g));
+              started[g] = true;
+              if (cur[g][0].head() < 0 && cur[g][1].head() < 0) f |= kLast0 << g;
+            }
+          }
+          if (!ok) {
+            wt.fail_check();
+            break;
+          }
+          const bool last = cur[0][0].head() < 0 && cur[0][1].head() < 0 && cur[1][0].head() < 0 &&
+                            cur[1][1].head() < 0;
+          if (last) f |= kItemLast;
+          ok = bundle(true, j, it.h, it.b, f);
+          if (last) break;
+          f = 0u;
+        }
+        }
+        live_pairs += uint32_t(it.n[0] + it.n[1] + it.n2[0] + it.n2[1]);
         ++qn;
       }
       ctl->tiles = live_pairs;
@@ -641,14 +712,16 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) ptx::mbar_arrive(BAR(item_empty[slot]));
       ++items;
       if (!ptx::named_bar_and(gbar, 128, ok) || it.row0 < 0) break;
-      const int qi = it.qt[grp];  // Tq when the item has no second query tile
-      const int n = it.n[grp];
-      const int row = it.row0 + qi;
+      const int qi = it.qt[grp];  // Tkq when the item has no second query tile
+      const int n = it.n[grp] + it.n2[grp];  // live tiles of the kernel query tile's mask rows
+      const int half = C::MR == 1 ? 0 : (r >> 6);  // stacked rows: which mask row this thread's row is in
+      const int row = it.row0 + qi * C::MR;         // first mask row of the kernel query tile
+      const int vrow = row + half;                  // this thread's mask row
       const int rq = r - grp * C::ROW1;  // row inside the query tile
       const int n_row = qi * C::BQ + rq;
-      const bool valid_row = qi < p.Tq && rq >= 0 && rq < C::BQ && n_row < p.Nq;
+      const bool valid_row = qi < p.Tkq && rq >= 0 && rq < C::BQ && n_row < p.Nq;
       const size_t o_off = (size_t(it.b) * p.Nq + n_row) * p.H + it.h;
-      const bool any = it.n[0] + it.n[1] > 0;
+      const bool any = it.n[0] + it.n[1] + it.n2[0] + it.n2[1] > 0;
       if (n == 0) {
         // a query tile without live key tiles: O = 0, lse = -inf; o_free keeps one phase per item
         if (valid_row) {
@@ -662,111 +735,150 @@ __global__ void __launch_bounds__(320, 1)
       float m_true = -INFINITY;  // running max over the tile's earlier live key tiles (log2 units)
       float m_used = -INFINITY;  // exponent reference (lazy rescale)
       float l = 0.f;             // row sum relative to m_used
-      int e_cur = it.e[grp][0], e_nxt = it.e[grp][1];
-      for (int idx = 0; idx < n; ++idx) {
-        const uint32_t t = tg + idx;
-        const int j = e_cur & kListIndexMask;
-        const bool may_flag = !(e_cur & kListNoFlag);
-        e_cur = e_nxt;
-        if (idx + 2 < n) e_nxt = key_entry(p, row, idx + 2);  // prefetch
-        if (r == 0) LITE_TRACE(2 + grp, 0, t);
-        // s_full[g] next completes for g's next live tile, whose QK follows this tile's PV
-        wt.wait(BAR(s_full[grp]), t & 1);
-        __syncwarp();
-        ptx::tc_fence_after();
-        float loc = -INFINITY;  // the tile's row max (log2 units)
-        if (!idle_warp) {
-        const uint32_t s_tmem = tmem + lane_base + C::S_COL + grp * BN;
-        // the whole S row is read once and stays in registers for the max and the exponentials
-        uint32_t sr[BN];
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c)
-          ptx::tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-        ptx::tmem_wait_ld();
-        if (r == 0) LITE_TRACE(2 + grp, 1, t);
-        float s[BN];
-#pragma unroll
-        for (int x = 0; x < BN; ++x) s[x] = __uint_as_float(sr[x]);
-        const int valid_cols = min(BN, p.Nk - j * BN);
-        if (valid_cols < BN) {
-          // key columns past Nk (zero-filled by TMA) take no part in max, sum or PV
-#pragma unroll
-          for (int x = 0; x < BN; ++x)
-            if (x >= valid_cols) s[x] = -INFINITY;
-        }
-        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-#pragma unroll
-        for (int x = 0; x < BN; x += 8) {
-          m0 = ptx::fmax3(m0, s[x], s[x + 1]);
-          m1 = ptx::fmax3(m1, s[x + 2], s[x + 3]);
-          m2 = ptx::fmax3(m2, s[x + 4], s[x + 5]);
-          m3 = ptx::fmax3(m3, s[x + 6], s[x + 7]);
-        }
-        loc = ptx::fmax3(m0, m1, fmaxf(m2, m3)) * p.scale_log2;
-        // lazy rescale of the accumulator: move the reference only when the tile max exceeds it by
-        // more than kRescaleLog2. O itself is rescaled after the exponentials below, when the S row
-        // no longer occupies registers (doing it here made the compiler spill S on every tile).
-        const bool need = loc > m_used + kRescaleLog2;
-        float alpha = 1.f;
-        if (need) {
-          alpha = ptx::ex2(m_used - loc);
-          m_used = loc;
-          l *= alpha;
-        }
-        // P = 2^(s*scale*log2e - m_used) as bf16 pairs over the S columns (chunk c of 32 key
-        // columns -> TMEM columns [16c, 16c+16)), released to the MMA thread in one piece. Packed
-        // fp32x2 arithmetic for the affine step and the row sum; one column pair in sixteen is
-        // exponentiated on the FMA pipe, the rest on MUFU (measured: 1/16 and none beat 1/8 and 1/4
-        // by ~1% once the O rescale left the S -> P path).
-        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-        const float2 nm2 = make_float2(-m_used, -m_used);
-        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const float2 a = __ffma2_rn(make_float2(s[32 * c + 2 * x], s[32 * c + 2 * x + 1]), sc2, nm2);
-            const float2 pp = (x == 15) ? exp2_poly2(a) : make_float2(ptx::ex2(a.x), ptx::ex2(a.y));
-            acc[x & 3] = __fadd2_rn(acc[x & 3], pp);
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(pp.x, pp.y);
-            pk[x] = *reinterpret_cast<uint32_t*>(&h2);
+      // One live key tile j of the kernel query tile (t counts the group's tiles over all items,
+      // idx within this item); live_me is false only for a stacked row whose mask row skips j.
+      auto tile = [&](uint32_t t, int j, bool may_flag, bool live_me, int idx) {
+          if (r == 0) LITE_TRACE(2 + grp, 0, t);
+          // s_full[g] next completes for g's next live tile, whose QK follows this tile's PV
+          wt.wait(BAR(s_full[grp]), t & 1);
+          __syncwarp();
+          ptx::tc_fence_after();
+          float loc = -INFINITY;  // the tile's row max (log2 units)
+          if (!idle_warp && !live_me) {
+            // (stacked rows only) key tile j is skipped for this row's mask row: P = 0 for the row
+            const uint32_t s_tmem = tmem + lane_base + C::S_COL + grp * BN;
+            uint32_t zero[16];
+  #pragma unroll
+            for (int x = 0; x < 16; ++x) zero[x] = 0u;
+  #pragma unroll
+            for (int c = 0; c < BN / 32; ++c) ptx::tmem_st16(s_tmem + c * 16, zero);
+            ptx::tmem_wait_st();
           }
-          ptx::tmem_st16(s_tmem + c * 16, pk);
-        }
-        // The previous PV into O_g was issued before this tile's QK, so it has completed now that S
-        // is ready; the rescaled O is stored before P is released (both stores are waited for below).
-        if (__any_sync(0xffffffffu, need) && idx >= 1) {
-          const uint32_t o_tmem = tmem + lane_base + C::O_COL + grp * D;
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t rr[32];
-            ptx::tmem_ld32(o_tmem + c * 32, rr);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int x = 0; x < 32; ++x) rr[x] = __float_as_uint(__uint_as_float(rr[x]) * alpha);
-            ptx::tmem_st32(o_tmem + c * 32, rr);
+          if (!idle_warp && live_me) {
+          const uint32_t s_tmem = tmem + lane_base + C::S_COL + grp * BN;
+          // the whole S row is read once and stays in registers for the max and the exponentials
+          uint32_t sr[BN];
+  #pragma unroll
+          for (int c = 0; c < BN / 32; ++c)
+            ptx::tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+          ptx::tmem_wait_ld();
+          if (r == 0) LITE_TRACE(2 + grp, 1, t);
+          float s[BN];
+  #pragma unroll
+          for (int x = 0; x < BN; ++x) s[x] = __uint_as_float(sr[x]);
+          const int valid_cols = min(BN, p.Nk - j * BN);
+          if (valid_cols < BN) {
+            // key columns past Nk (zero-filled by TMA) take no part in max, sum or PV
+  #pragma unroll
+            for (int x = 0; x < BN; ++x)
+              if (x >= valid_cols) s[x] = -INFINITY;
           }
+          float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+  #pragma unroll
+          for (int x = 0; x < BN; x += 8) {
+            m0 = ptx::fmax3(m0, s[x], s[x + 1]);
+            m1 = ptx::fmax3(m1, s[x + 2], s[x + 3]);
+            m2 = ptx::fmax3(m2, s[x + 4], s[x + 5]);
+            m3 = ptx::fmax3(m3, s[x + 6], s[x + 7]);
+          }
+          loc = ptx::fmax3(m0, m1, fmaxf(m2, m3)) * p.scale_log2;
+          // lazy rescale of the accumulator: move the reference only when the tile max exceeds it by
+          // more than kRescaleLog2. O itself is rescaled after the exponentials below, when the S row
+          // no longer occupies registers (doing it here made the compiler spill S on every tile).
+          const bool need = loc > m_used + kRescaleLog2;
+          float alpha = 1.f;
+          if (need) {
+            alpha = ptx::ex2(m_used - loc);
+            m_used = loc;
+            l *= alpha;
+          }
+          // P = 2^(s*scale*log2e - m_used) as bf16 pairs over the S columns (chunk c of 32 key
+          // columns -> TMEM columns [16c, 16c+16)), released to the MMA thread in one piece. Packed
+          // fp32x2 arithmetic for the affine step and the row sum; one column pair in sixteen is
+          // exponentiated on the FMA pipe, the rest on MUFU (measured: 1/16 and none beat 1/8 and 1/4
+          // by ~1% once the O rescale left the S -> P path).
+          const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+          const float2 nm2 = make_float2(-m_used, -m_used);
+          float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  #pragma unroll
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t pk[16];
+  #pragma unroll
+            for (int x = 0; x < 16; ++x) {
+              const float2 a = __ffma2_rn(make_float2(s[32 * c + 2 * x], s[32 * c + 2 * x + 1]), sc2, nm2);
+              const float2 pp = (x == 15) ? exp2_poly2(a) : make_float2(ptx::ex2(a.x), ptx::ex2(a.y));
+              acc[x & 3] = __fadd2_rn(acc[x & 3], pp);
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(pp.x, pp.y);
+              pk[x] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            ptx::tmem_st16(s_tmem + c * 16, pk);
+          }
+          // The previous PV into O_g was issued before this tile's QK, so it has completed now that S
+          // is ready; the rescaled O is stored before P is released (both stores are waited for below).
+          if (__any_sync(0xffffffffu, need) && idx >= 1) {
+            const uint32_t o_tmem = tmem + lane_base + C::O_COL + grp * D;
+  #pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t rr[32];
+              ptx::tmem_ld32(o_tmem + c * 32, rr);
+              ptx::tmem_wait_ld();
+  #pragma unroll
+              for (int x = 0; x < 32; ++x) rr[x] = __float_as_uint(__uint_as_float(rr[x]) * alpha);
+              ptx::tmem_st32(o_tmem + c * 32, rr);
+            }
+          }
+          ptx::tmem_wait_st();
+          const float2 acc2 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+          l += acc2.x + acc2.y;
+          }
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(BAR(p_full[grp]));
+          if (r == 0) LITE_TRACE(2 + grp, 2, t);
+          if (p.skip_test && live_me) {
+            // QK-Skip, off the path from S to P: flag key tile j when loc - m < tau for every valid
+            // row of the mask row, m the running max over the row's earlier live key tiles. With
+            // stacked rows each 64-row half votes on its own named barrier (its two warps).
+            const bool pred = !valid_row || (loc - m_true < p.tau_log2);
+            const bool flag = C::MR == 1 ? ptx::named_bar_and(gbar, 128, pred)
+                                         : ptx::named_bar_and(3 + 2 * grp + half, 64, pred);
+            if (flag && may_flag && (r & (C::BM / C::MR - 1)) == 0 && p.mask_out && !ctl->abort)
+              atomicOr(p.mask_out + size_t(vrow) * p.W + (j >> 5), 1u << (j & 31));
+          }
+          if (r == 0) LITE_TRACE(2 + grp, 3, t);
+          m_true = fmaxf(m_true, loc);
+      };
+      if constexpr (C::MR == 1) {
+        int e_cur = it.e[grp][0], e_nxt = it.e[grp][1];
+        for (int idx = 0; idx < n; ++idx) {
+          const int j = e_cur & kListIndexMask;
+          const bool may_flag = !(e_cur & kListNoFlag);
+          e_cur = e_nxt;
+          if (idx + 2 < n) e_nxt = key_entry(p, row, idx + 2);  // prefetch
+          tile(tg + idx, j, may_flag, true, idx);
         }
-        ptx::tmem_wait_st();
-        const float2 acc2 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-        l += acc2.x + acc2.y;
+        tg += n;
+      } else {
+        // the union of the kernel query tile's two mask rows' lists, highest key tile first
+        const int mi = half, oi = 1 - half;
+        const int nm = mi == 0 ? it.n[grp] : it.n2[grp], no = oi == 0 ? it.n[grp] : it.n2[grp];
+        ListCursor mine{row + mi, nm, 0, mi == 0 ? it.e[grp][0] : it.e2[grp][0], mi == 0 ? it.e[grp][1] : it.e2[grp][1],
+                        p.Tk};
+        ListCursor other{row + oi, no, 0, oi == 0 ? it.e[grp][0] : it.e2[grp][0], oi == 0 ? it.e[grp][1] : it.e2[grp][1],
+                         p.Tk};
+        int idx = 0;
+        while (true) {
+          const int hm = mine.head(), ho = other.head();
+          if (hm < 0 && ho < 0) break;
+          const int j = max(hm, ho);
+          const bool live_me = hm == j;
+          const bool may_flag = live_me && !(mine.cur & kListNoFlag);
+          if (live_me) mine.advance(p);
+          if (ho == j) other.advance(p);
+          tile(tg + idx, j, may_flag, live_me, idx);
+          ++idx;
         }
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(BAR(p_full[grp]));
-        if (r == 0) LITE_TRACE(2 + grp, 2, t);
-        if (p.skip_test) {
-          // QK-Skip, off the path from S to P: flag key tile j when loc - m < tau for every valid
-          // row, m the running max over the tile's earlier live key tiles
-          const bool pred = !valid_row || (loc - m_true < p.tau_log2);
-          const bool flag = ptx::named_bar_and(gbar, 128, pred);
-          if (flag && may_flag && r == 0 && p.mask_out && !ctl->abort)
-            atomicOr(p.mask_out + size_t(row) * p.W + (j >> 5), 1u << (j & 31));
-        }
-        if (r == 0) LITE_TRACE(2 + grp, 3, t);
-        m_true = fmaxf(m_true, loc);
+        tg += idx;
       }
-      tg += n;
       // Epilogue: wait for the item's last PV into O_g, normalise, and write the rows (bf16) out
       // through shared memory: each warp stages the rows of lanes 0-15, then those of lanes 16-31,
       // and its lane 0 issues one TMA store per half (rows past Nq are clipped by the TMA unit). A
@@ -775,7 +887,8 @@ __global__ void __launch_bounds__(320, 1)
       wt.wait(BAR(pv_done[grp]), pv_phase & 1);
       ++pv_phase;
       ptx::tc_fence_after();
-      const float inv_l = 1.f / l;
+      // a stacked row whose mask row has no live tile in the item: O = 0, lse = -inf
+      const float inv_l = (C::MR == 1 || l > 0.f) ? 1.f / l : 0.f;
       uint32_t ow[D / 2];  // the row's D columns, packed in bf16 pairs
 #pragma unroll
       for (int c = 0; c < D / 32 && !idle_warp; ++c) {
@@ -809,14 +922,15 @@ __global__ void __launch_bounds__(320, 1)
           ptx::fence_proxy_async_smem();
           __syncwarp();
           const int row_in_tile = wrow + half * C::OST_ROWS;
-          if (lane == 0 && qi < p.Tq && row_in_tile < C::BQ && qi * C::BQ + row_in_tile < p.Nq) {
+          if (lane == 0 && qi < p.Tkq && row_in_tile < C::BQ && qi * C::BQ + row_in_tile < p.Nq) {
             ptx::tma_store_5d(&tmO, ptx::smem_addr(stage), 0, qi * C::BQ + row_in_tile, 0, it.h, it.b);
             ptx::bulk_commit_group();
           }
         }
       }
       if (valid_row && p.lse)
-        p.lse[(size_t(it.b) * p.H + it.h) * p.Nq + n_row] = (m_used + __log2f(l)) * 0.6931471805599453f;
+        p.lse[(size_t(it.b) * p.H + it.h) * p.Nq + n_row] =
+            (C::MR == 1 || l > 0.f) ? (m_used + __log2f(l)) * 0.6931471805599453f : -INFINITY;
     }
     // the staged O rows must have been written out before the CTA (and its shared memory) ends
     if (lane == 0) ptx::bulk_wait_group0();

@@ -115,6 +115,9 @@ bool debug_env() {
 
 int tile_for(int d) { return d == 64 ? 64 : (d == 128 ? 128 : 0); }
 
+// Skip-Mask rows stacked in one 128-row kernel query tile: 2 for the 64-row tiles of d = 64.
+int mask_rows_per_tile(int d) { return 128 / tile_for(d); }
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_shapes(int B, int H, int Nq, int Nk, int d) {
@@ -202,8 +205,9 @@ lite::AttnParams base_params(void* o, float* lse, int B, int H, int Nq, int Nk, 
   p.Tq = (Nq + t - 1) / t;
   p.Tk = (Nk + t - 1) / t;
   p.W = (p.Tk + 31) / 32;
-  p.Pq = (p.Tq + 1) / 2;
-  p.n_items = B * H * p.Pq;  // work items: pairs of query tiles
+  p.Tkq = (p.Tq + mask_rows_per_tile(d) - 1) / mask_rows_per_tile(d);  // kernel query tiles of 128 rows
+  p.Pq = (p.Tkq + 1) / 2;
+  p.n_items = B * H * p.Pq;  // work items: pairs of kernel query tiles
   p.pair_stride = 1;
   p.scale_log2 = resolve_scale(scale, d) * 1.4426950408889634f;
   p.tau_log2 = -INFINITY;
@@ -270,8 +274,11 @@ int enqueue_pairs(const FwdArgs& a, const uint32_t* mask_in, const int32_t* coun
                   lite::AttnParams& p, cudaStream_t s) {
   const Tail t = tail_at(tail);
   const int Tq = p.Tq, BH = a.B * a.H;
+  const bool stacked = mask_rows_per_tile(a.d) == 2;
+  // The stride is scored for one mask row per kernel query tile (d = 128); with stacked rows
+  // (d = 64) the kernel query tiles are paired consecutively unless the option fixes a stride.
   const int n_cand = std::max(1, std::min(lite::kMaxPairStride, Tq / 2));
-  const bool scored = g_opt.pair_stride == 0 && mask_in != nullptr && n_cand > 1;
+  const bool scored = !stacked && g_opt.pair_stride == 0 && mask_in != nullptr && n_cand > 1;
   if (scored) {
     const int chunks = std::max(1, std::min(8, BH));
     lite::lite_stride_score_kernel<<<dim3(n_cand, chunks), 256, 0, s>>>(mask_in, t.scores, BH, Tq, p.Tk, p.W);
@@ -279,8 +286,12 @@ int enqueue_pairs(const FwdArgs& a, const uint32_t* mask_in, const int32_t* coun
   }
   if (g_opt.schedule) {
     const size_t sm = size_t(BH + p.Pq) * sizeof(int32_t);
-    lite::lite_schedule_kernel<2><<<BH, 512, sm, s>>>(counts, order, BH, Tq, scored ? t.scores : nullptr, n_cand,
-                                                      g_opt.pair_stride, t.stride);
+    if (stacked)
+      lite::lite_schedule_kernel<4><<<BH, 512, sm, s>>>(counts, order, BH, Tq, nullptr, 0, g_opt.pair_stride,
+                                                        t.stride);
+    else
+      lite::lite_schedule_kernel<2><<<BH, 512, sm, s>>>(counts, order, BH, Tq, scored ? t.scores : nullptr, n_cand,
+                                                        g_opt.pair_stride, t.stride);
     if (cudaGetLastError() != cudaSuccess) return LITE_ERR_CUDA;
     p.pair_stride_ptr = t.stride;  // written by the schedule kernel
   } else {

@@ -200,7 +200,10 @@ __device__ __forceinline__ int pick_stride(const uint32_t* scores, int n_cand, i
 // smem: totals[BH] ints, then counts of this head [T] ints
 // G = 1 orders the query tiles of every head; G = 2 orders pairs of query tiles (pair_tiles with the
 // picked stride, which CTA 0 also writes to *stride_out), the work items of the attention kernel, by
-// their combined live count. Output entries are head * ceil(T/G) + item.
+// their combined live count; G = 4 orders the work items of the stacked-row attention kernel (d = 64:
+// a pair of 128-row kernel query tiles, each two mask rows), by the live count of their four mask
+// rows, consecutive kernel tiles assumed (the stride written is the option's, else 1). Output
+// entries are head * ceil(T/G) + item.
 template <int G>
 __global__ void __launch_bounds__(512) lite_schedule_kernel(const int32_t* __restrict__ counts,
                                                            int32_t* __restrict__ order, int BH, int T,
@@ -211,8 +214,8 @@ __global__ void __launch_bounds__(512) lite_schedule_kernel(const int32_t* __res
   int32_t* totals = sh;
   int32_t* mine = sh + BH;
   const int g = blockIdx.x;
-  const int stride = G == 2 ? pick_stride(scores, n_cand, fixed_stride) : 1;
-  if (G == 2 && g == 0 && threadIdx.x == 0 && stride_out) *stride_out = stride;
+  const int stride = G >= 2 ? pick_stride(scores, n_cand, fixed_stride) : 1;
+  if (G >= 2 && g == 0 && threadIdx.x == 0 && stride_out) *stride_out = stride;
   for (int x = threadIdx.x; x < BH; x += blockDim.x) totals[x] = 0;
   __syncthreads();
   // per-head totals (every CTA computes all of them; B*H*T ints, served from L2)
@@ -221,13 +224,15 @@ __global__ void __launch_bounds__(512) lite_schedule_kernel(const int32_t* __res
     if (v) atomicAdd(&totals[x / T], v);
   }
   for (int x = threadIdx.x; x < P; x += blockDim.x) {
-    int c;
+    int c = 0;
     if constexpr (G == 2) {
       int a, b;
       pair_tiles(x, T, stride, a, b);
       c = __ldg(counts + size_t(g) * T + a) + (b >= 0 ? __ldg(counts + size_t(g) * T + b) : 0);
     } else {
-      c = __ldg(counts + size_t(g) * T + x);
+#pragma unroll
+      for (int k = 0; k < G; ++k)
+        if (G * x + k < T) c += __ldg(counts + size_t(g) * T + G * x + k);
     }
     mine[x] = c;
   }
