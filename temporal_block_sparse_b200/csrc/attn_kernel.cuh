@@ -1,15 +1,17 @@
 // attn_kernel.cuh -- persistent block-sparse attention forward for sm_100a (tcgen05 + TMEM + TMA).
 //
-// One CTA per SM walks a list of work items; an item is a pair of query tiles of one (b, h): tile r
-// and tile r + s of each block of 2s tiles, with the pairing stride s chosen per call as the one
-// whose pairs share the most live key tiles (s = 28 on 720p-like layers, one latent frame apart). For each query tile it computes only the live key tiles of that tile
-// (LiteAttention README, "Full-Stage Elimination": a skipped tile costs no K/V load, no QK^T, no
-// softmax, no PV), from the highest key-tile index down (README, must_do_list: "we iterate in
-// reverse order inside of the kernel"). The two query tiles share K/V: the CTA walks the union of
-// their two Skip-Lists, loads each union tile once, and computes it for the query tiles it is live
-// for. Queries and keys may differ in length (README, LSE section: partial attentions such as
-// text-to-video over a subset of the keys); a key tile that a must-do range keeps live carries a
-// tag in its list entry and is computed but never flagged.
+// One CTA per SM walks a list of work items; an item is a pair of 128-row query tiles of one
+// (b, h): tile r and tile r + s of each block of 2s tiles, with the pairing stride s chosen per call
+// as the one whose pairs share the most live key tiles (s = 28 on 720p-like layers, one latent frame
+// apart). With d = 64 a 128-row query tile stacks two 64-row Skip-Mask rows, each with its own list.
+// For each query tile it computes only the live key tiles of that tile (LiteAttention README,
+// "Full-Stage Elimination": a skipped tile costs no K/V load, no QK^T, no softmax, no PV), from the
+// highest key-tile index down (README, must_do_list: "we iterate in reverse order inside of the
+// kernel"). The two query tiles share K/V: the CTA walks the union of their Skip-Lists, loads each
+// union tile once, and computes it for the query tiles it is live for. Queries and keys may differ
+// in length (README, LSE section: partial attentions such as text-to-video over a subset of the
+// keys); a key tile that a must-do range keeps live carries a tag in its list entry and is computed
+// but never flagged.
 //
 // Warp roles (320 threads):
 //   warp 0       TMA producer: per item the pair's two Q tiles; per union tile u a load bundle with
@@ -103,8 +105,7 @@ struct AttnCfg {
   // QK-Skip vote; a key tile live for only one half computes the other half's rows too and gives
   // them P = 0.
   static constexpr int MR = BM / BN;             // mask rows per kernel query tile: 1 (d=128), 2 (d=64)
-  static constexpr int BQ = BM;                  // query rows per kernel query tile
-  static constexpr int ROW1 = BM - BQ;           // 0: both query-tile slots are full
+  static constexpr int BQ = BM;                  // query rows per kernel query tile (both slots full)
   static constexpr int THREADS = 320;            // producer warp, MMA warp, 2 softmax warpgroups
   static constexpr int NCHUNK = D / 64;          // 128-byte swizzle atoms along d
   static constexpr int Q_CHUNK = BM * 128;       // bytes between d-chunks of a Q tile in smem
@@ -413,16 +414,6 @@ __global__ void __launch_bounds__(320, 1)
     ptx::prefetch_tmap(&tmV);
     ptx::prefetch_tmap(&tmO);
   }
-  if constexpr (C::BQ < C::BM) {
-    // Q rows outside the query tile are never loaded; keep them zero so their S rows stay finite.
-    for (int g = 0; g < 2; ++g)
-      for (int c = 0; c < C::NCHUNK; ++c) {
-        const int zrow = g == 0 ? C::BQ : 0;  // the rows of slot g that hold no query row
-        uint4* z = reinterpret_cast<uint4*>(smem + C::OFF_Q + g * C::Q_BYTES + c * C::Q_CHUNK + zrow * 128);
-        for (int x = threadIdx.x; x < (C::BM - C::BQ) * 128 / 16; x += blockDim.x) z[x] = make_uint4(0, 0, 0, 0);
-      }
-    ptx::fence_proxy_async_smem();
-  }
   if (warp == 1) {
     ptx::tmem_alloc(ptx::smem_addr(&ctl->tmem_base), C::TMEM_COLS);
     ptx::tmem_relinquish();
@@ -512,8 +503,7 @@ __global__ void __launch_bounds__(320, 1)
         ptx::mbar_arrive_expect_tx(BAR(q_full), (gn[0] > 0 ? C::Q_TX : 0u) + (gn[1] > 0 ? C::Q_TX : 0u));
         for (int g = 0; g < 2; ++g)
           if (gn[g] > 0)
-            ptx::tma_load_5d(sQ + g * C::Q_BYTES + g * C::ROW1 * 128, &tmQ, BAR(q_full), 0, it.qt[g] * C::BQ, 0, it.h,
-                             it.b);
+            ptx::tma_load_5d(sQ + g * C::Q_BYTES, &tmQ, BAR(q_full), 0, it.qt[g] * C::BQ, 0, it.h, it.b);
         q_armed = true;
         q_par = qn & 1;
         const uint32_t item_bits = ((qn & 1) ? kItemOdd : 0u) | (qn >= 1 ? kItemAfterFirst : 0u);
@@ -699,10 +689,7 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
     const uint32_t gbar = 1 + grp;                  // named barrier of this warpgroup (128 threads)
     uint8_t* stage = smem + C::OFF_OST + (grp * 4 + quarter) * C::OST_WARP;
-    // a warp whose 32 lanes hold no row of its group's query tile (64-row tiles only) keeps the
-    // group's barrier sequence but does no TMEM, exponential or store work
-    const int wrow = quarter * 32 - grp * C::ROW1;
-    const bool idle_warp = C::ROW1 > 0 && (wrow < 0 || wrow >= C::BQ);
+    const int wrow = quarter * 32;                  // first tile row of this warp's lanes
     uint32_t tg = 0, items = 0, pv_phase = 0;
     while (true) {
       const int slot = items & 1;
@@ -717,7 +704,7 @@ __global__ void __launch_bounds__(320, 1)
       const int half = C::MR == 1 ? 0 : (r >> 6);  // stacked rows: which mask row this thread's row is in
       const int row = it.row0 + qi * C::MR;         // first mask row of the kernel query tile
       const int vrow = row + half;                  // this thread's mask row
-      const int rq = r - grp * C::ROW1;  // row inside the query tile
+      const int rq = r;  // row inside the kernel query tile
       const int n_row = qi * C::BQ + rq;
       const bool valid_row = qi < p.Tkq && rq >= 0 && rq < C::BQ && n_row < p.Nq;
       const size_t o_off = (size_t(it.b) * p.Nq + n_row) * p.H + it.h;
@@ -744,7 +731,7 @@ __global__ void __launch_bounds__(320, 1)
           __syncwarp();
           ptx::tc_fence_after();
           float loc = -INFINITY;  // the tile's row max (log2 units)
-          if (!idle_warp && !live_me) {
+          if (!live_me) {
             // (stacked rows only) key tile j is skipped for this row's mask row: P = 0 for the row
             const uint32_t s_tmem = tmem + lane_base + C::S_COL + grp * BN;
             uint32_t zero[16];
@@ -754,7 +741,7 @@ __global__ void __launch_bounds__(320, 1)
             for (int c = 0; c < BN / 32; ++c) ptx::tmem_st16(s_tmem + c * 16, zero);
             ptx::tmem_wait_st();
           }
-          if (!idle_warp && live_me) {
+          if (live_me) {
           const uint32_t s_tmem = tmem + lane_base + C::S_COL + grp * BN;
           // the whole S row is read once and stays in registers for the max and the exponentials
           uint32_t sr[BN];
@@ -891,7 +878,7 @@ __global__ void __launch_bounds__(320, 1)
       const float inv_l = (C::MR == 1 || l > 0.f) ? 1.f / l : 0.f;
       uint32_t ow[D / 2];  // the row's D columns, packed in bf16 pairs
 #pragma unroll
-      for (int c = 0; c < D / 32 && !idle_warp; ++c) {
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t rr[32];
         ptx::tmem_ld32(tmem + lane_base + C::O_COL + grp * D + c * 32, rr);
         ptx::tmem_wait_ld();
@@ -904,28 +891,26 @@ __global__ void __launch_bounds__(320, 1)
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(BAR(o_free[grp]));
-      if (!idle_warp) {
-        const int srow = lane & (C::OST_ROWS - 1);
+      const int srow = lane & (C::OST_ROWS - 1);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          if (lane == 0) ptx::bulk_wait_group_read0();
-          __syncwarp();
-          if ((lane >> 4) == half) {
+      for (int part = 0; part < 2; ++part) {
+        if (lane == 0) ptx::bulk_wait_group_read0();
+        __syncwarp();
+        if ((lane >> 4) == part) {
 #pragma unroll
-            for (int c = 0; c < D / 8; ++c) {
-              // 16-byte chunk c of the row: panel c/8, 128-byte swizzle (chunk ^ row % 8) inside it
-              const int x = c & 7;
-              *reinterpret_cast<uint4*>(stage + (c >> 3) * C::OST_PANEL + srow * 128 + ((x ^ (srow & 7)) << 4)) =
-                  make_uint4(ow[4 * c], ow[4 * c + 1], ow[4 * c + 2], ow[4 * c + 3]);
-            }
+          for (int c = 0; c < D / 8; ++c) {
+            // 16-byte chunk c of the row: panel c/8, 128-byte swizzle (chunk ^ row % 8) inside it
+            const int x = c & 7;
+            *reinterpret_cast<uint4*>(stage + (c >> 3) * C::OST_PANEL + srow * 128 + ((x ^ (srow & 7)) << 4)) =
+                make_uint4(ow[4 * c], ow[4 * c + 1], ow[4 * c + 2], ow[4 * c + 3]);
           }
-          ptx::fence_proxy_async_smem();
-          __syncwarp();
-          const int row_in_tile = wrow + half * C::OST_ROWS;
-          if (lane == 0 && qi < p.Tkq && row_in_tile < C::BQ && qi * C::BQ + row_in_tile < p.Nq) {
-            ptx::tma_store_5d(&tmO, ptx::smem_addr(stage), 0, qi * C::BQ + row_in_tile, 0, it.h, it.b);
-            ptx::bulk_commit_group();
-          }
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        const int row_in_tile = wrow + part * C::OST_ROWS;
+        if (lane == 0 && qi < p.Tkq && row_in_tile < C::BQ && qi * C::BQ + row_in_tile < p.Nq) {
+          ptx::tma_store_5d(&tmO, ptx::smem_addr(stage), 0, qi * C::BQ + row_in_tile, 0, it.h, it.b);
+          ptx::bulk_commit_group();
         }
       }
       if (valid_row && p.lse)
