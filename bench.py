@@ -542,7 +542,9 @@ def main():
             "dense_path_tflops": layer_dense_flop / (dense_ms_step * 1e-3) / 1e12,
             "roofline": roofline,
             "mask_kernels": mask_roof,
-            "gpu_launches": 3 * args.steps,
+            # per step: compaction, pairing-stride scores (d = 128 with more than two query tiles),
+            # schedule, attention
+            "gpu_launches": (4 if d == 128 and T // 2 > 1 else 3) * args.steps,
             "clocks": clock_info,
             "steady": steady,
             "e2e": e2e,

@@ -131,8 +131,8 @@ int lite_mask_to_ranges(const uint32_t* mask, int16_t* ranges, int32_t* nruns, i
 
 /*
  * lite_schedule -- longest-first order of query tiles (no counterpart on the pages). The
- * attention kernel behind lite_attn_fwd takes its work in pairs of consecutive query tiles (2i,
- * 2i+1) of one head and orders those pairs the same way, by their combined live count.
+ * attention kernel behind lite_attn_fwd takes its work in pairs of query tiles of one head (see
+ * LITE_OPT_PAIR_STRIDE) and orders those pairs the same way, by their combined live count.
  *
  * Heads (b, h) are ordered by decreasing total live-tile count (ties: lower b*H+h first); inside a
  * head, query tiles by decreasing live count (ties: lower index first). Writes order[B*H*T] with

@@ -156,9 +156,10 @@ def test_optional_outputs_and_no_mask():
 
 @pytest.mark.parametrize("d,gw", [(64, 15), (128, 14)])
 def test_paired_query_tiles_with_disjoint_lists(d, gw):
-    """The kernel pairs query tiles (2i, 2i+1) and walks the union of their Skip-Lists. Here the
-    two tiles of each pair have disjoint live sets: even key tiles for one, odd for the other, so
-    every union tile is live for one query tile only. One pair has a fully skipped tile, and an
+    """The kernel pairs query tiles and walks the union of their Skip-Lists; with d = 64 each
+    128-row kernel tile stacks two 64-row mask rows. Here neighbouring query tiles have disjoint
+    live sets: even key tiles for one, odd for the other, so most union tiles (and, at d = 64,
+    every key tile of a stacked pair of rows) are live for one query tile only. One pair has a fully skipped tile, and an
     odd tile count leaves the last query tile without a partner. All rows against the oracle,
     three steps with QK-Skip on."""
     tile = 64 if d == 64 else 128
@@ -327,28 +328,56 @@ def _mask_bits(mask, T):
     return np.unpackbits(mask.cpu().numpy().view(np.uint8), axis=-1, bitorder="little")[..., :T].astype(bool)
 
 
+def _pairing_partner(live):
+    """The partner of every query tile under the pairing the kernel picks for this mask: the stride
+    s in [1, min(64, T/2)] whose pairs (tile r with r + s inside each block of 2s tiles, the tiles
+    after the last full block as (t, t+1)) share the most live key tiles, the smaller on ties
+    (include/lite_attn.h, LITE_OPT_PAIR_STRIDE). Returns partner[T] (-1: no partner)."""
+    B, H, T, _ = live.shape
+    X = live.astype(np.int64)
+
+    def pairs(s):
+        full = (T // (2 * s)) * (2 * s)
+        idx = np.arange(full)
+        a = idx[(idx % (2 * s)) < s]
+        rest = np.arange(full, T - 1, 2)
+        return np.concatenate([a, rest]), np.concatenate([a + s, rest + 1])
+
+    best, best_s = -1, 1
+    for s in range(1, max(1, min(64, T // 2)) + 1):
+        a, b = pairs(s)
+        sc = int((X[:, :, a] & X[:, :, b]).sum())
+        if sc > best:
+            best, best_s = sc, s
+    a, b = pairs(best_s)
+    partner = np.full(T, -1)
+    partner[a], partner[b] = b, a
+    return partner
+
+
 def _lone_heavy_tiles(skipped, n, seed):
-    """Query tiles whose pair partner (2i, 2i+1 share a CTA) has a disjoint or empty live list, so
-    that the kernel's union walk gives them many key tiles computed for one query tile only; the
-    first and the ragged last tile of a head are always included."""
+    """Query tiles whose pair partner (under the pairing the kernel picks) has a disjoint or empty
+    live list, so that the kernel's union walk gives them many key tiles computed for one query
+    tile only; the first and the ragged last tile of a head are always included."""
     B, H, T, _ = skipped.shape
     live = ~skipped
-    partner = np.arange(T) ^ 1
-    has_partner = partner < T
+    partner = _pairing_partner(live)
+    has_partner = partner >= 0
+    pidx = np.where(has_partner, partner, 0)
     own = live.sum(-1)
-    shared = np.where(has_partner, (live & live[:, :, np.minimum(partner, T - 1)]).sum(-1), 0)
+    shared = np.where(has_partner, (live & live[:, :, pidx]).sum(-1), 0)
     lone = own - shared  # live tiles of this query tile that its partner skips
     rng = np.random.default_rng(seed)
     picks = {(0, 0, 0), (B - 1, H - 1, T - 1)}
     if (~has_partner).any():
-        picks.add((0, int(rng.integers(H)), T - 1))  # an unpaired last tile
+        picks.add((0, int(rng.integers(H)), int(np.argmin(has_partner))))  # an unpaired tile
     order = np.argsort(-(lone + rng.random(lone.shape)), axis=None)  # most lone tiles first, ties random
     for flat in order[: 4 * n]:
         b, h, i = np.unravel_index(flat, lone.shape)
         picks.add((int(b), int(h), int(i)))
         if len(picks) >= n - 2:
             break
-    empty_partner = np.argwhere((own > 0) & has_partner & (own[:, :, np.minimum(partner, T - 1)] == 0))
+    empty_partner = np.argwhere((own > 0) & has_partner & (own[:, :, pidx] == 0))
     for b, h, i in empty_partner[:2]:
         picks.add((int(b), int(h), int(i)))
     while len(picks) < n:
