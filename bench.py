@@ -918,7 +918,7 @@ def _load_balance(la, q, k, v, mask, tau):
     """Per-CTA busy time of the attention kernel on one mask, with the longest-first schedule and with
     query tiles in their natural order: {order: {kernel_ms, busy max/mean, tiles max/mean}}."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    buf = torch.zeros((sms, 3), dtype=torch.int64, device="cuda")
+    buf = torch.zeros((2 * sms, 3), dtype=torch.int64, device="cuda")  # up to two CTAs per SM
     m_out = torch.empty_like(mask)
     out = {}
     for name, sched in (("longest_first", 1), ("natural", 0)):

@@ -167,7 +167,8 @@ const char* lite_status_string(int status);
  *                          kernel gives up and reports LITE_ERR_TIMEOUT (default 4e9; >= 1000).
  *  LITE_OPT_DEBUG_STALL    1 = test hook: the MMA warp of every CTA withholds its first tile, so
  *                          the waits that depend on it run out their limit (no fault, no hang).
- *  LITE_OPT_MAX_CTAS       cap on the persistent grid size (0 = one CTA per SM).
+ *  LITE_OPT_MAX_CTAS       cap on the persistent grid size (0 = every resident CTA slot: one
+ *                          CTA per SM with d = 128, two per SM with d = 64).
  *  LITE_OPT_SCHEDULE       1 (default) = lite_attn_fwd* hand out their work items (pairs of
  *                          query tiles of one head, see LITE_OPT_PAIR_STRIDE) longest first, heads
  *                          kept together, as lite_schedule orders query tiles; 0 = in their

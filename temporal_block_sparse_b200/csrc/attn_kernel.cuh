@@ -1,6 +1,7 @@
 // attn_kernel.cuh -- persistent block-sparse attention forward for sm_100a (tcgen05 + TMEM + TMA).
 //
-// One CTA per SM walks a list of work items; an item is a pair of 128-row query tiles of one
+// Persistent CTAs (one per SM with d = 128; two per SM with d = 64, whose CTA needs half the TMEM
+// columns) walk a list of work items; an item is a pair of 128-row query tiles of one
 // (b, h): tile r and tile r + s of each block of 2s tiles, with the pairing stride s chosen per call
 // as the one whose pairs share the most live key tiles (s = 28 on 720p-like layers, one latent frame
 // apart). With d = 64 a 128-row query tile stacks two 64-row Skip-Mask rows, each with its own list.
@@ -126,13 +127,21 @@ struct AttnCfg {
   static constexpr int OST_WARP = NCHUNK * OST_PANEL;
   static constexpr int OFF_OST = (OFF_CTL + CTL_BYTES + 1023) / 1024 * 1024;
   static constexpr int OST_BYTES = 8 * OST_WARP;
-  // one CTA per SM: the request is padded so that two never fit (TMEM is sized for one)
   static constexpr int SMEM_USED = OFF_OST + OST_BYTES + 1024;
-  static constexpr int SMEM_BYTES = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   // TMEM columns: S_0 [0, BN), S_1 [BN, 2BN), O_0 [2BN, 2BN+D), O_1 [2BN+D, 2BN+2D)
   static constexpr uint32_t S_COL = 0;
   static constexpr uint32_t O_COL = 2 * BN;
   static constexpr uint32_t TMEM_COLS = (2 * BN + 2 * D) <= 256 ? 256 : 512;
+  // Resident CTAs per SM. A CTA holds TMEM_COLS of the SM's 512 TMEM columns for its whole life.
+  // With d = 64 that is 256, so two CTAs run side by side (96 registers a thread, ~83 KB of shared
+  // memory each) and hide each other's per-tile latencies. With d = 128 a CTA takes all 512
+  // columns, and its shared-memory request is padded so that a second CTA can never be placed
+  // on the SM and block in its TMEM allocation.
+  static constexpr int CTAS_PER_SM = int(512 / TMEM_COLS);
+  static constexpr int SMEM_BYTES =
+      CTAS_PER_SM == 2 ? SMEM_USED : (SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024);
+  // two CTAs (each also reserving 1 KB of shared memory) within the SM's 228 KB
+  static_assert(CTAS_PER_SM == 1 || 2 * (SMEM_BYTES + 1024) <= 228 * 1024, "two CTAs per SM");
   // instruction descriptors, kind::f16: fp32 accumulate (bit 4), bf16 A (bits 7-9) and B (10-12),
   // B major-ness (bit 16), N >> 3 (bits 17-22), M >> 4 (bits 24-28)
   static constexpr uint32_t IDESC_QK = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) |
@@ -375,7 +384,7 @@ constexpr float kRescaleLog2 = 2.0f;
 constexpr uint32_t kItemOdd = 512u, kItemAfterFirst = 1024u;
 
 template <int D, int BN>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(320, AttnCfg<D, BN>::CTAS_PER_SM)
     lite_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                      const AttnParams p) {

@@ -174,7 +174,7 @@ int launch_attention(DeviceCache* dc, int cfg_slot, const void* q, const void* k
   if (!make_tmap(&tq, q, p.B, p.Nq, p.H, D, C::BQ) || !make_tmap(&tk, k, p.B, p.Nk, p.H, D, BN) ||
       !make_tmap(&tv, v, p.B, p.Nk, p.H, D, BN) || !make_tmap(&to, p.o, p.B, p.Nq, p.H, D, C::OST_ROWS))
     return LITE_ERR_CUDA;
-  int grid = dc->sms;
+  int grid = dc->sms * C::CTAS_PER_SM;  // persistent: every resident CTA slot
   if (g_opt.max_ctas > 0 && g_opt.max_ctas < grid) grid = g_opt.max_ctas;
   if (p.n_items < grid) grid = p.n_items;
   if (grid <= 0) return LITE_OK;
