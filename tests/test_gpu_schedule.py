@@ -72,6 +72,30 @@ def test_cta_timing_counts_every_live_tile():
     assert int(rec[used, 2].sum()) == live
 
 
+def test_head_dim_64_runs_two_ctas_per_sm():
+    """With d = 64 a CTA holds half of the SM's TMEM columns, so the persistent grid has two CTAs
+    per SM and they run side by side: every CTA takes work, the CTAs start together (not in two
+    waves), and their tiles add up to the layer's."""
+    w = wl.small_workload(1, 8, 8, 32, 64, 64, locality=2.0, seed_offset=64)  # N = 16384, 512 items
+    q, k, v = wl.Trajectory(w, device="cuda").current()
+    B, N, H, d = q.shape
+    _, T, _ = la.lite_mask_geometry(N, d)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    buf = torch.zeros((2 * sms + 8, 3), dtype=torch.int64, device="cuda")
+    la.lite_set_cta_timing(buf)
+    la.lite_attn_fwd(q, k, v, None, None, tau=-3.0)
+    torch.cuda.synchronize()
+    la.lite_set_cta_timing(None)
+    rec = buf.cpu().numpy()
+    used = rec[:, 1] > 0
+    assert used.sum() == 2 * sms
+    assert (rec[used, 2] > 0).all()
+    assert int(rec[used, 2].sum()) == B * H * T * T  # no mask: every tile is live
+    starts, ends = rec[used, 0], rec[used, 1]
+    # a second wave would start only when the first CTAs ran out of work
+    assert starts.max() - starts.min() < 0.25 * (ends.max() - starts.min())
+
+
 def _run_with(q, k, v, m_in, tau, **opts):
     for name, val in opts.items():
         la.lite_set_option(getattr(la, name), val)
