@@ -510,7 +510,7 @@ def main():
     roofline = {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
                 "frac": achieved / burst, "traffic": traffic,
                 "peak_kind": f"{peak_src} dense bf16 cuBLAS, burst (sustained under the power cap: {sustained})",
-                "frac_of_sustained": achieved / sustained, "kernel": "lite_attn_kernel<128,128>",
+                "frac_of_sustained": achieved / sustained, "kernel": f"lite_attn_kernel<{d},{tile}>",
                 "flop_per_launch": flop_per_launch,
                 "attn_ms_per_launch": attn_avg_ms, "attn_share_of_step": sum(attn_ms) / elapsed_ms}
 

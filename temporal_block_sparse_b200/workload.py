@@ -74,6 +74,8 @@ WORKLOADS = {
     "tiny": Workload("tiny", 1, 1, 4, 16, 16, 64, 5, 2.0, 0.05, _tau_const(-3.0), seed_offset=1),
     # one layer at a 480p-like latent (21 frames x 30x52), tau linear -10 -> 0 over 10 steps
     "480p": Workload("480p", 1, 40, 21, 30, 52, 128, 10, 2.0, 0.05, _tau_linear(-10.0, 0.0), seed_offset=2),
+    # the 480p latent at head dimension 64 (tile 64), tau=-3, 10 steps
+    "480p_d64": Workload("480p_d64", 1, 40, 21, 30, 52, 64, 10, 2.0, 0.05, _tau_const(-3.0), seed_offset=6),
     # one layer at a Wan2.1-14B 720p-like latent (21 frames x 45x80), tau=-3, 50 steps, 3% drift
     "720p": Workload("720p", 1, 40, 21, 45, 80, 128, 50, 3.0, 0.03, _tau_const(-3.0), seed_offset=3),
     # threshold sweep on the 720p shape (tau fixed per run, set by the caller), 20 steps
