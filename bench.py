@@ -73,11 +73,19 @@ def parse_args():
 # ----------------------------------------------------------------------------------------- helpers
 
 
+def code_text(src: str) -> str:
+    """C++ source without its comments and blank space, so that a comment edit keeps the hash."""
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
 def kernel_sha() -> str:
+    """Hash of the attention kernel's code (comments excluded), recorded with every ncu summary."""
     h = hashlib.sha256()
     for p in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, p), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, p), encoding="utf-8") as f:
+            h.update(code_text(f.read()).encode())
     return h.hexdigest()[:16]
 
 

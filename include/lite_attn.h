@@ -58,7 +58,7 @@ enum {
  * mask_in leaves live (README, "Full-Stage Elimination"), and lse = log-sum-exp of those scores
  * (README: LSE is returned for combining partial attentions). While doing so it runs the QK-Skip
  * test on every computed tile: the key tiles of a query tile are visited from the highest index
- * down (README, must_do_list: "we iterate in reverse order inside of the kernel"); with m_r the
+ * down (README, must_do_list: the kernel walks key positions in reverse order); with m_r the
  * running row maximum of scale*QK^T over the tiles visited before tile j and loc_r the row maximum
  * inside tile j, tile j is flagged when loc_r - m_r < tau for every valid row r of the query tile.
  * mask_out = mask_in | flags (README, "QK-Skip Algorithm": the number of skipped tiles only grows).
@@ -90,7 +90,8 @@ int lite_attn_fwd(const void* q, const void* k, const void* v, void* o, float* l
                   float scale, float tau, lite_stream_t stream);
 
 /*
- * lite_attn_dense -- the no-skip path (README: turning skipping off "falls back to regular FA3").
+ * lite_attn_dense -- the no-skip path (README, enable_skip_optimization: with skipping off the
+ * library runs plain FlashAttention-3).
  *
  * Same kernel and layouts as lite_attn_fwd with every tile live and the QK-Skip test off; no mask
  * is read or written and no scratch memory is allocated. lse may be NULL.
@@ -99,8 +100,9 @@ int lite_attn_dense(const void* q, const void* k, const void* v, void* o, float*
                     int N, int d, float scale, lite_stream_t stream);
 
 /*
- * lite_mask_to_list -- Skip-Mask to Skip-List compaction (skill page, Architecture Overview:
- * "Bitmask (or Skip-List for high sparsity)"; README: key ranges are iterated in reverse order).
+ * lite_mask_to_list -- Skip-Mask to Skip-List compaction (skill page, Architecture Overview: the
+ * skip state is a bitmask, or a list where sparsity is high; README: key ranges are walked in
+ * reverse order).
  *
  *  mask    in   device uint32 [B, H, T, W], or NULL = nothing skipped.
  *  list    out  device int16 [B, H, T, T]: for each (b, h, query tile) the live key tiles in
@@ -113,7 +115,7 @@ int lite_mask_to_list(const uint32_t* mask, int16_t* list, int32_t* counts, int 
 
 /*
  * lite_mask_to_ranges -- Skip-Mask to range-encoded Skip-List (skill page, Architecture Overview:
- * "Bitmask (or Skip-List for high sparsity)"; range pairs as in the README's must_do_list: start
+ * a bitmask, or a list where sparsity is high; range pairs as in the README's must_do_list: start
  * inclusive, end exclusive, strictly descending, because key tiles are visited in reverse order).
  *
  * For each (b, h, query tile), every maximal run of live key tiles a..b (a <= b, tile indices)
@@ -256,9 +258,9 @@ int lite_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
  * lite_attn_fwd_list -- lite_attn_fwd over caller-supplied Skip-Lists instead of a Skip-Mask.
  *
  * The skill page "Lite Attention Temporal Sparse" (Architecture Overview) keeps the skip state as a
- * bitmask "or Skip-List for high sparsity": per (b, h, query tile) the live key tiles, which the
- * kernel visits from the highest index down (README, must_do_list: "we iterate in reverse order
- * inside of the kernel"). lite_attn_fwd builds these lists from the mask (lite_mask_to_list) on every
+ * bitmask, or as a list where sparsity is high: per (b, h, query tile) the live key tiles, which
+ * the kernel visits from the highest index down (README, must_do_list: key positions are walked in
+ * reverse order). lite_attn_fwd builds these lists from the mask (lite_mask_to_list) on every
  * call; a caller that keeps the lists itself passes them here, and the compaction step and the mask
  * copy are skipped. Results are those of lite_attn_fwd on the mask the lists describe.
  *

@@ -10,7 +10,7 @@ Sources (the LiteAttention pages):
     iteration is bypassed at the following timesteps.
   * Same README, contribution list, "Full-Stage Elimination": a skipped tile costs no QK product, no
     softmax and no PV product.
-  * Same README, must_do_list convention: "we iterate in reverse order inside of the kernel", i.e.
+  * Same README, must_do_list convention: the kernel walks key positions in reverse order, i.e.
     the key tiles of a query tile are visited from the highest index down.
   * Same README, Python API: thresholds are negative log-domain numbers (default -10; -6, -3 and 0
     in the examples and the threshold ablation table); thresholds above 0 are a debug-only setting.
@@ -99,7 +99,7 @@ def live_key_tiles(mask: Optional[np.ndarray], b: int, h: int, i: int, T: int) -
 
 def visit_order(tiles) -> List[int]:
     """Order in which a query tile's live key tiles are visited: highest index first (README,
-    must_do_list: "we iterate in reverse order inside of the kernel")."""
+    must_do_list: the kernel walks key positions in reverse order)."""
     return sorted(tiles, reverse=True)
 
 

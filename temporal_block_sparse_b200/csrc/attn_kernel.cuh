@@ -7,8 +7,8 @@
 // apart). With d = 64 a 128-row query tile stacks two 64-row Skip-Mask rows, each with its own list.
 // For each query tile it computes only the live key tiles of that tile (LiteAttention README,
 // "Full-Stage Elimination": a skipped tile costs no K/V load, no QK^T, no softmax, no PV), from the
-// highest key-tile index down (README, must_do_list: "we iterate in reverse order inside of the
-// kernel"). The two query tiles share K/V: the CTA walks the union of their Skip-Lists, loads each
+// highest key-tile index down (README, must_do_list: the kernel walks key tiles in reverse
+// order). The two query tiles share K/V: the CTA walks the union of their Skip-Lists, loads each
 // union tile once, and computes it for the query tiles it is live for. Queries and keys may differ
 // in length (README, LSE section: partial attentions such as text-to-video over a subset of the
 // keys); a key tile that a must-do range keeps live carries a tag in its list entry and is computed

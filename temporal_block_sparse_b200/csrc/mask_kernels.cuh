@@ -97,8 +97,9 @@ __global__ void __launch_bounds__(256) lite_compact_kernel(const uint32_t* mask_
 }
 
 // Skip-Mask -> range-encoded Skip-List ("Lite Attention Temporal Sparse" skill page, Architecture
-// Overview: "Bitmask (or Skip-List for high sparsity)"; README must_do_list convention for ranges:
-// pairs (start inclusive, end exclusive) in strictly descending order, iterated in reverse).
+// Overview: the skip state is a bitmask, or a list where sparsity is high; README must_do_list
+// convention for ranges: pairs (start inclusive, end exclusive) in strictly descending order,
+// walked from the top down).
 // A run of live key tiles a..b (a <= b) becomes the pair (b, a - 1). One warp per (b, h, query
 // tile), words from the top down, lane l owns key tile 32w + 31 - l. A live tile opens a run when
 // the tile above it is not live and closes one when the tile below is not live; ballots of both
