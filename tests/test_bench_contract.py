@@ -97,3 +97,14 @@ def test_mask_kernel_bytes():
     rows = 2 * 40 * 591
     assert bench.mask_bytes(m, 1000, 591, with_copy=False) == rows * 19 * 4 + 2000 + rows * 4
     assert bench.mask_bytes(m, 1000, 591, with_copy=True) == 2 * rows * 19 * 4 + 2000 + rows * 4
+
+
+def test_kernel_hash_ignores_comments_only():
+    """The hash that ties a stored DRAM-traffic figure to the code it was captured on survives a
+    comment edit and changes with any edit to the code."""
+    import bench
+    code = "int f(int x) {\n  // the input, doubled\n  return 2 * x; /* twice */\n}\n"
+    recommented = "/* f doubles its input */\nint f(int x) {\n  return 2 * x;   // same code\n}\n"
+    changed = "int f(int x) {\n  return 3 * x;\n}\n"
+    assert bench.code_text(code) == bench.code_text(recommented)
+    assert bench.code_text(code) != bench.code_text(changed)
