@@ -293,6 +293,13 @@ def test_480p_layer_sampled_late_steps():
     assert sp[-1] > 0
 
 
+def test_480p_d64_layer_sampled():
+    """The 480p latent at d = 64: 512 mask rows stacked two to a kernel query tile, run by two
+    CTAs per SM; sampled mask rows over three steps of its trajectory."""
+    sp = _full_size("480p_d64", 3, 12)
+    assert sp[-1] > 0
+
+
 @pytest.mark.parametrize("d,F,gh,gw", [(64, 27, 133, 73), (128, 5, 47, 2231)])
 def test_maximum_tile_count(d, F, gh, gw):
     """The largest layer the library accepts: 4096 query and key tiles (N = 262,143 at d=64 and
