@@ -22,6 +22,7 @@ def _clean_state():
     yield
     la.lite_set_option(la.LITE_OPT_SCHEDULE, 1)
     la.lite_set_option(la.LITE_OPT_PAIR_STRIDE, 0)
+    la.lite_set_option(la.LITE_OPT_MAX_CTAS, 0)
     la.lite_set_cta_timing(None)
     assert la.lite_get_device_status() == 0
 
@@ -94,6 +95,27 @@ def test_head_dim_64_runs_two_ctas_per_sm():
     starts, ends = rec[used, 0], rec[used, 1]
     # a second wave would start only when the first CTAs ran out of work
     assert starts.max() - starts.min() < 0.25 * (ends.max() - starts.min())
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_grid_size_gives_identical_results(d):
+    """Every work item computes the same bits whichever CTA takes it: the full grid (two CTAs per
+    SM at d = 64), an odd cap that leaves some SMs one CTA, and a single CTA."""
+    w = wl.small_workload(1, 16, 8, 32, 32, d, steps=2, locality=4.0, tau=-2.0, seed_offset=70 + d)  # 512 items
+    tr = wl.Trajectory(w, device="cuda")
+    q, k, v = tr.current()
+    B, N, H, _ = q.shape
+    m0 = la.new_mask(B, H, N, d)
+    m_in = torch.empty_like(m0)
+    la.lite_attn_fwd(q, k, v, m0, m_in, tau=-2.0)  # a grown, uneven mask for the compared step
+    tr.advance()
+    q, k, v = tr.current()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    runs = [_run_with(q, k, v, m_in, -2.0, LITE_OPT_MAX_CTAS=cap) for cap in (0, sms + 1, 1)]
+    la.lite_set_option(la.LITE_OPT_MAX_CTAS, 0)
+    for other in runs[1:]:
+        for a, b in zip(runs[0], other):
+            assert torch.equal(a, b)
 
 
 def _run_with(q, k, v, m_in, tau, **opts):
